@@ -1,0 +1,230 @@
+"""fp64 CPU oracle for sink-aware sliding-window attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline and reference legs may import this package.  The CUDA
+library never calls it, imports nothing from it and shares no code with it.
+
+The arithmetic lives in ``swa_oracle.c`` (plain C, double precision, OpenMP
+over query rows); this module only marshals numpy arrays through ctypes and
+holds the plain model of the ring-buffer KV cache (slot bookkeeping, no
+arithmetic on values).
+
+Parity pins: every function here is checked by the ``-m "not gpu"`` tests
+against closed forms, a library causal-attention routine, brute-force masks
+built from the set definition, and hand-derived golden values.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "swa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+_lib_path = _LIB
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile swa_oracle.c into liboracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def use_library(path: str) -> None:
+    """Point the wrappers at another build of swa_oracle.c (the tests use this to
+    show that a deliberately broken copy fails the pins)."""
+    global _lib, _lib_path
+    with _lock:
+        _lib, _lib_path = None, path
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            if _lib_path == _LIB:
+                build()
+            lib = ctypes.CDLL(_lib_path)
+            lib.oracle_swa_rows.argtypes = [_dp, _i64p, ctypes.c_int64, _dp, _dp, ctypes.c_int64,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                            ctypes.c_int64, ctypes.c_double, _dp, _dp, ctypes.c_int]
+            lib.oracle_swa_weights.argtypes = [_dp, ctypes.c_int64, _dp, ctypes.c_int64, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                               ctypes.c_int64, ctypes.c_double, _dp]
+            lib.oracle_swa_fwd.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+            lib.oracle_swa_fwd_varlen.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64p, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                                  ctypes.c_int]
+            lib.oracle_visible_count.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+            lib.oracle_visible_count.restype = ctypes.c_int64
+            lib.oracle_num_threads.argtypes = [ctypes.c_int]
+            for f in (lib.oracle_swa_rows, lib.oracle_swa_weights, lib.oracle_swa_fwd,
+                      lib.oracle_swa_fwd_varlen, lib.oracle_num_threads):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact float64 copy of a numpy array or a (CPU or CUDA) torch tensor."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_dp)
+
+
+def num_threads(n: int = 0) -> int:
+    """Threads the oracle's OpenMP loops use (n > 0 sets it)."""
+    return _load().oracle_num_threads(int(n))
+
+
+def visible_count(t: int, window: int, n_sink: int) -> int:
+    return int(_load().oracle_visible_count(int(t), int(window), int(n_sink)))
+
+
+def swa_rows(q_rows, t_rows, k, v, window: int, n_sink: int, scale: float, threads: int = 0):
+    """Selected rows of one sequence.
+
+    q_rows [n, Hq, d]; t_rows [n] positions; k, v [L, Hkv, d].
+    Returns out [n, Hq, d] and lse [n, Hq] (float64).
+    """
+    q = _f64(q_rows)
+    k = _f64(k)
+    v = _f64(v)
+    t = np.ascontiguousarray(np.asarray(t_rows, dtype=np.int64))
+    n, Hq, d = q.shape
+    L, Hkv, _ = k.shape
+    out = np.zeros((n, Hq, d))
+    lse = np.zeros((n, Hq))
+    rc = _load().oracle_swa_rows(_p(q), t.ctypes.data_as(_i64p), n, _p(k), _p(v), L, Hq, Hkv, d,
+                                 int(window), int(n_sink), float(scale), _p(out), _p(lse),
+                                 int(threads))
+    if rc != 0:
+        raise ValueError("oracle_swa_rows rejected its arguments")
+    return out, lse
+
+
+def swa_weights(q_row, t: int, k, h: int, window: int, n_sink: int, scale: float):
+    """Attention weights over keys 0..L-1 of query head h at row t; q_row [Hq, d], k [L, Hkv, d]."""
+    q = _f64(q_row)
+    k = _f64(k)
+    Hq, d = q.shape
+    L, Hkv, _ = k.shape
+    w = np.zeros(L)
+    rc = _load().oracle_swa_weights(_p(q), int(t), _p(k), L, Hq, Hkv, d, int(h), int(window),
+                                    int(n_sink), float(scale), _p(w))
+    if rc != 0:
+        raise ValueError("oracle_swa_weights rejected its arguments")
+    return w
+
+
+def swa_fwd(q, k, v, window: int, n_sink: int, scale: float, threads: int = 0):
+    """q [B, L, Hq, d], k/v [B, L, Hkv, d] -> out [B, L, Hq, d], lse [B, Hq, L] (float64)."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    out = np.zeros_like(q)
+    lse = np.zeros((B, Hq, L))
+    rc = _load().oracle_swa_fwd(_p(q), _p(k), _p(v), _p(out), _p(lse), B, Hq, Hkv, L, d,
+                                int(window), int(n_sink), float(scale), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_swa_fwd rejected its arguments")
+    return out, lse
+
+
+def swa_fwd_varlen(q, k, v, cu_seqlens, window: int, n_sink: int, scale: float, threads: int = 0):
+    """Packed q [T, Hq, d], k/v [T, Hkv, d], cu_seqlens [n+1] -> out [T, Hq, d], lse [Hq, T]."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    out = np.zeros_like(q)
+    lse = np.zeros((Hq, T))
+    rc = _load().oracle_swa_fwd_varlen(_p(q), _p(k), _p(v), _p(out), _p(lse),
+                                       cu.ctypes.data_as(_i64p), len(cu) - 1, Hq, Hkv, d,
+                                       int(window), int(n_sink), float(scale), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_swa_fwd_varlen rejected its arguments")
+    return out, lse
+
+
+def swa_decode(q, k_hist, v_hist, pos, window: int, n_sink: int, scale: float, threads: int = 0):
+    """Decode by definition: row t = pos[b] of sequence b, whose keys/values at
+    positions 0..pos[b] are k_hist[b, :pos[b]+1] (k_hist/v_hist [B, P, Hkv, d]).
+
+    q [B, Hq, d] -> out [B, Hq, d], lse [B, Hq].
+    """
+    q = _f64(q)
+    B, Hq, d = q.shape
+    out = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        p = int(pos[b])
+        o, l_ = swa_rows(q[b:b + 1], [p], k_hist[b, :p + 1], v_hist[b, :p + 1], window, n_sink,
+                         scale, threads)
+        out[b], lse[b] = o[0], l_[0]
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Ring-buffer KV cache model (slot bookkeeping only).
+#
+# "Sliding-window beats linear attention", section 1: sliding-window attention
+# keeps a fixed-size memory at inference, and the first tokens (sinks) must
+# stay.  Reading used throughout: position p lives in ring slot p mod w; the
+# positions p < n_sink are also kept in pinned sink slot p and are never
+# evicted.  Writing position p overwrites (evicts) position p - w.
+# ---------------------------------------------------------------------------
+
+def ring_fill(k, v, window: int, n_sink: int):
+    """Cache contents after positions 0..P-1 of k/v [B, P, Hkv, d] were written.
+
+    Returns kcache, vcache [B, Hkv, window, d] and sink_k, sink_v [B, Hkv, n_sink, d]
+    (numpy, same dtype as the input; untouched slots are zero).
+    """
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, P, Hkv, d = k.shape
+    kc = np.zeros((B, Hkv, window, d), dtype=k.dtype)
+    vc = np.zeros_like(kc)
+    sk = np.zeros((B, Hkv, n_sink, d), dtype=k.dtype)
+    sv = np.zeros_like(sk)
+    for p in range(P):
+        ring_append(kc, vc, sk, sv, k[:, p], v[:, p], np.full(B, p), window, n_sink)
+    return kc, vc, sk, sv
+
+
+def ring_append(kc, vc, sk, sv, k_new, v_new, pos, window: int, n_sink: int) -> None:
+    """In place: write position pos[b] (k_new/v_new [B, Hkv, d]) into the cache arrays."""
+    for b in range(len(pos)):
+        p = int(pos[b])
+        kc[b, :, p % window] = k_new[b]
+        vc[b, :, p % window] = v_new[b]
+        if p < n_sink:
+            sk[b, :, p] = k_new[b]
+            sv[b, :, p] = v_new[b]
