@@ -1,0 +1,170 @@
+/*
+ * libswa — causal sliding-window softmax attention with attention sinks on
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes, no framework types.
+ *
+ * The operation ("Sliding-window beats linear attention", section 1 Key Terms
+ * and section 3): query position t of a sequence attends to the keys
+ *     S(t) = { j : j <= t  and  ( j >= t - window + 1  or  j < n_sink ) },
+ * i.e. a causal window of `window` keys ending at t plus the first `n_sink`
+ * positions of its sequence (the attention sinks), which stay visible at every
+ * position; a key that is both is counted once.  With G = Hq / Hkv, query head
+ * h reads KV head h / G (grouped-query attention, "Rethinking Attention Output
+ * Projection", section 1).  For each (t, h):
+ *     z_j = scale * <q_t,h , k_j,kvh>,  out = softmax_j(z) . v,  lse = ln sum_j exp(z_j).
+ *
+ * Conventions shared by every entry point:
+ *   - Every device pointer is owned by the caller, must stay valid until the
+ *     work queued on `stream` has finished, and must be 16-byte aligned.
+ *     The library allocates no device memory and keeps no device state except
+ *     one error word per device (see swa_device_error).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  The return value reports argument errors
+ *     (nothing launched) and launch errors only; a device-side wait that ran
+ *     past its time limit is reported through swa_device_error.
+ *   - bf16 is IEEE bfloat16 stored as uint16; f32 is IEEE binary32.
+ *   - Accumulation is fp32.  In the bf16 path the softmax numerators P are
+ *     rounded to bf16 (round-to-nearest-even) before the P.V product and the
+ *     output is rounded to bf16; the fp32 path runs both products as tf32.
+ */
+#ifndef SWA_H
+#define SWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* swa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  SWA_OK = 0,
+  SWA_ERR_INVALID_ARG = 1,    /* a size, pointer or alignment precondition failed; nothing launched */
+  SWA_ERR_UNSUPPORTED = 2,    /* valid arguments outside what the kernels implement (e.g. d = 96) */
+  SWA_ERR_CUDA = 3,           /* the CUDA runtime or driver reported an error */
+  SWA_ERR_DEVICE_TIMEOUT = 4, /* a kernel gave up on a barrier wait (swa_device_error only) */
+  SWA_ERR_WORKSPACE = 5       /* workspace pointer missing or smaller than required */
+} swa_status;
+
+/* Element types of q, k, v / out. */
+typedef enum {
+  SWA_DTYPE_BF16 = 0,         /* bf16 in, bf16 out */
+  SWA_DTYPE_F32 = 1,          /* f32 in, f32 out (products run as tf32) */
+  SWA_DTYPE_BF16_F32OUT = 2   /* bf16 in, f32 out (same arithmetic as SWA_DTYPE_BF16, no final rounding) */
+} swa_dtype;
+
+/*
+ * Prefill over B sequences of equal length L.
+ *   q   [B, L, Hq, d]    input type     (row-major, contiguous)
+ *   k,v [B, L, Hkv, d]   input type
+ *   out [B, L, Hq, d]    output type    (written)
+ *   lse [B, Hq, L]       float32        (written; may be NULL)
+ * Requires Hq % Hkv == 0, window >= 1, n_sink >= 0, scale > 0 and finite.
+ * Supported: bf16 inputs (either output type) with d in {64, 128}; f32 with d = 64.
+ * Nothing is launched (and SWA_OK returned) when B * L == 0.
+ */
+int swa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+            int B, int Hq, int Hkv, int L, int d, int window, int n_sink, float scale,
+            int dtype, swa_stream_t stream);
+
+/*
+ * Prefill over n_seq packed sequences of different lengths; sequence i owns
+ * tokens cu_seqlens[i] .. cu_seqlens[i+1]-1 and its window and sinks are
+ * counted from its own first token.
+ *   q   [T, Hq, d], k,v [T, Hkv, d] (input type), out [T, Hq, d] (output type)
+ *   lse [Hq, T]      float32 (may be NULL)
+ *   cu_seqlens       DEVICE int32 [n_seq + 1], non-decreasing, cu_seqlens[0] = 0,
+ *                    cu_seqlens[n_seq] = T (not checked: the device reads it)
+ * Requires 1 <= n_seq <= 1024 and the same head/dtype preconditions as swa_fwd.
+ */
+int swa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                   const int32_t* cu_seqlens, int n_seq, long long T,
+                   int Hq, int Hkv, int d, int window, int n_sink, float scale,
+                   int dtype, swa_stream_t stream);
+
+/*
+ * Ring-buffer KV cache for decoding ("Sliding-window beats linear attention",
+ * section 1: sliding-window attention needs a fixed amount of memory at
+ * inference; section 3: the sinks must be kept).  Layout, all bf16:
+ *   kcache, vcache  [B, Hkv, window, d]   position p lives in slot p mod window
+ *   sink_k, sink_v  [B, Hkv, n_sink, d]   position p < n_sink also lives in sink slot p
+ * Writing position p overwrites slot p mod window, which evicts position
+ * p - window.  Sink slots are written once and never evicted.
+ */
+
+/*
+ * Fill an empty cache with the prefix positions 0 .. P-1 of k, v [B, P, Hkv, d]
+ * (bf16).  Only the last min(P, window) positions reach the ring and only
+ * positions < n_sink reach the sink slots.  sink_k/sink_v may be NULL when
+ * n_sink == 0.  P == 0 launches nothing.
+ */
+int swa_cache_fill(const void* k, const void* v, int P,
+                   void* kcache, void* vcache, void* sink_k, void* sink_v,
+                   int B, int Hkv, int d, int window, int n_sink, swa_stream_t stream);
+
+/*
+ * Append one token per sequence: k_new, v_new [B, Hkv, d] (bf16) are written at
+ * position pos[b] (DEVICE int32 [B], pos[b] >= 0) into slot pos[b] mod window,
+ * and into sink slot pos[b] when pos[b] < n_sink.
+ */
+int swa_cache_append(const void* k_new, const void* v_new, const int32_t* pos,
+                     void* kcache, void* vcache, void* sink_k, void* sink_v,
+                     int B, int Hkv, int d, int window, int n_sink, swa_stream_t stream);
+
+/*
+ * Bytes of device workspace swa_decode needs for these sizes (fp32 split
+ * partials).  Pure host function; 0 means the sizes are invalid.
+ */
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int window, int n_sink);
+
+/*
+ * One decode step: query q [B, Hq, d] (bf16) of position pos[b] attends to the
+ * cached keys of S(pos[b]): ring slots holding positions max(0, pos-window+1)
+ * .. pos and the sink slots j < min(n_sink, pos - window + 1).  The caller must
+ * have appended position pos[b] (and every earlier one) before this call.
+ *   out [B, Hq, d] bf16 (written), lse [B, Hq] float32 (written; may be NULL)
+ *   workspace: device buffer of at least swa_decode_workspace_bytes(...) bytes,
+ *   256-byte aligned; contents need not be initialised and are scratch.
+ * The keys are split evenly over the GPU's warps (split-K); the partial
+ * softmax states are merged by their log-sum-exps in a second kernel.
+ * Supported: d in {64, 128}, Hq / Hkv <= 8.
+ */
+int swa_decode(const void* q, const void* kcache, const void* vcache,
+               const void* sink_k, const void* sink_v, const int32_t* pos,
+               void* out, float* lse,
+               int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
+               void* workspace, size_t workspace_bytes, swa_stream_t stream);
+
+/* Static text for a status code. */
+const char* swa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error
+ * word: SWA_OK, or SWA_ERR_DEVICE_TIMEOUT when a kernel abandoned a barrier
+ * wait after the time limit (it then wrote no output and released its tensor
+ * memory).  Returns SWA_ERR_CUDA if the synchronisation itself failed.
+ */
+int swa_device_error(swa_stream_t stream);
+
+/*
+ * Time limit, in nanoseconds, of every device-side barrier wait launched after
+ * this call (default 2e9).  Process-wide.  Returns the previous value.
+ */
+unsigned long long swa_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * Test hook, process-wide: flags = 1 makes the prefill kernel's load warp
+ * issue no copies, so that its consumers' bounded waits run out.  0 restores
+ * normal operation.  Returns the previous flags.
+ */
+int swa_set_debug_flags(int flags);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int swa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H */

@@ -1,0 +1,201 @@
+"""Python binding of libswa (causal sliding-window attention with attention sinks, B200).
+
+Argument marshalling only: every function passes raw device pointers, sizes
+and the current CUDA stream to the C ABI declared in ``include/swa.h``; all of
+the work runs in the library's sm_100a kernels.  There is no fallback: if
+``libswa.so`` is missing or cannot be loaded, every call raises.
+
+Tensors are PyTorch tensors on a CUDA device (PyTorch only supplies memory and
+streams).  Layouts follow ``swa.h``:
+    prefill      q [B, L, Hq, d], k/v [B, L, Hkv, d], out like q, lse [B, Hq, L]
+    varlen       q [T, Hq, d], k/v [T, Hkv, d], cu_seqlens int32 [n+1], lse [Hq, T]
+    ring cache   kcache/vcache [B, Hkv, window, d], sink_k/sink_v [B, Hkv, n_sink, d]
+    decode       q [B, Hq, d], pos int32 [B], out [B, Hq, d], lse [B, Hq]
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libswa.so")
+
+SWA_OK = 0
+SWA_ERR_INVALID_ARG = 1
+SWA_ERR_UNSUPPORTED = 2
+SWA_ERR_CUDA = 3
+SWA_ERR_DEVICE_TIMEOUT = 4
+SWA_ERR_WORKSPACE = 5
+SWA_DTYPE_BF16 = 0
+SWA_DTYPE_F32 = 1
+SWA_DTYPE_BF16_F32OUT = 2
+
+# Every entry point of include/swa.h.
+EXPORTS = (
+    "swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append",
+    "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
+    "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version",
+)
+
+_lib = None
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {swa_status_string(status)} (status {status})")
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with `python -m sink_aware_sliding_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_size_t
+    lib.swa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_fwd_varlen.argtypes = [P, P, P, P, P, P, I, LL, I, I, I, I, I, F, I, P]
+    lib.swa_cache_fill.argtypes = [P, P, I, P, P, P, P, I, I, I, I, I, P]
+    lib.swa_cache_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
+    lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.swa_decode_workspace_bytes.restype = SZ
+    lib.swa_decode.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_status_string.argtypes = [I]
+    lib.swa_status_string.restype = ctypes.c_char_p
+    lib.swa_device_error.argtypes = [P]
+    lib.swa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+    lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
+    lib.swa_set_debug_flags.argtypes = [I]
+    for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
+                 "swa_device_error", "swa_set_debug_flags", "swa_version"):
+        getattr(lib, name).restype = I
+    _lib = lib
+    return lib
+
+
+def library():
+    """The loaded ctypes library (raises if libswa.so is missing)."""
+    return _load()
+
+
+def _check(st: int, where: str) -> None:
+    if st != SWA_OK:
+        raise SwaError(st, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t, out) -> int:
+    import torch
+    if t.dtype == torch.bfloat16 and out.dtype == torch.bfloat16:
+        return SWA_DTYPE_BF16
+    if t.dtype == torch.bfloat16 and out.dtype == torch.float32:
+        return SWA_DTYPE_BF16_F32OUT
+    if t.dtype == torch.float32 and out.dtype == torch.float32:
+        return SWA_DTYPE_F32
+    raise TypeError(f"unsupported dtypes {t.dtype} -> {out.dtype}")
+
+
+def _scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def swa_status_string(status: int) -> str:
+    return _load().swa_status_string(int(status)).decode()
+
+
+def swa_version() -> int:
+    return _load().swa_version()
+
+
+def swa_fwd(q, k, v, out, lse, window: int, n_sink: int, scale=None, stream=None) -> None:
+    """Prefill; q [B, L, Hq, d], k/v [B, L, Hkv, d]; writes out (like q) and lse [B, Hq, L] (or None)."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape and out.shape == q.shape, "shapes")
+    _need(all(t.is_contiguous() for t in (q, k, v, out)), "tensors must be contiguous")
+    _need(q.dtype == k.dtype == v.dtype, "q, k, v must share a dtype")
+    B, L, Hq, d = q.shape
+    _need(k.shape[0] == B and k.shape[1] == L and k.shape[3] == d, "k/v shape")
+    if lse is not None:
+        _need(lse.shape == (B, Hq, L) and lse.is_contiguous(), "lse shape")
+    st = _load().swa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, k.shape[2], L, d,
+                         int(window), int(n_sink), _scale(scale, d), _dtype_code(q, out), _stream(stream))
+    _check(st, "swa_fwd")
+
+
+def swa_fwd_varlen(q, k, v, out, lse, cu_seqlens, window: int, n_sink: int, scale=None,
+                   stream=None) -> None:
+    """Packed prefill; q [T, Hq, d], k/v [T, Hkv, d], cu_seqlens int32 [n+1] on the device."""
+    _need(q.dim() == 3 and k.dim() == 3 and v.shape == k.shape and out.shape == q.shape, "shapes")
+    _need(all(t.is_contiguous() for t in (q, k, v, out, cu_seqlens)), "tensors must be contiguous")
+    import torch
+    _need(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1, "cu_seqlens must be int32 [n+1]")
+    T, Hq, d = q.shape
+    if lse is not None:
+        _need(lse.shape == (Hq, T) and lse.is_contiguous(), "lse shape")
+    st = _load().swa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+                                cu_seqlens.numel() - 1, T, Hq, k.shape[1], d, int(window),
+                                int(n_sink), _scale(scale, d), _dtype_code(q, out), _stream(stream))
+    _check(st, "swa_fwd_varlen")
+
+
+def swa_cache_fill(k, v, kcache, vcache, sink_k, sink_v, window: int, n_sink: int,
+                   stream=None) -> None:
+    """Write prefix positions 0..P-1 of k/v [B, P, Hkv, d] into an empty ring cache."""
+    B, P, Hkv, d = k.shape
+    st = _load().swa_cache_fill(_ptr(k), _ptr(v), P, _ptr(kcache), _ptr(vcache), _ptr(sink_k),
+                                _ptr(sink_v), B, Hkv, d, int(window), int(n_sink), _stream(stream))
+    _check(st, "swa_cache_fill")
+
+
+def swa_cache_append(k_new, v_new, pos, kcache, vcache, sink_k, sink_v, window: int, n_sink: int,
+                     stream=None) -> None:
+    """Write k_new/v_new [B, Hkv, d] at positions pos (int32 [B], device) into the ring cache."""
+    B, Hkv, d = k_new.shape
+    st = _load().swa_cache_append(_ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(kcache), _ptr(vcache),
+                                  _ptr(sink_k), _ptr(sink_v), B, Hkv, d, int(window), int(n_sink),
+                                  _stream(stream))
+    _check(st, "swa_cache_append")
+
+
+def swa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, window: int, n_sink: int) -> int:
+    return int(_load().swa_decode_workspace_bytes(B, Hq, Hkv, d, window, n_sink))
+
+
+def swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,
+               workspace, scale=None, stream=None) -> None:
+    """One decode step; q [B, Hq, d] bf16 at positions pos; writes out [B, Hq, d] and lse [B, Hq]."""
+    B, Hq, d = q.shape
+    Hkv = kcache.shape[1]
+    st = _load().swa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(sink_k), _ptr(sink_v),
+                            _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window), int(n_sink),
+                            _scale(scale, d), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream))
+    _check(st, "swa_decode")
+
+
+def swa_device_error(stream=None) -> int:
+    return _load().swa_device_error(_stream(stream))
+
+
+def swa_set_wait_timeout_ns(ns: int) -> int:
+    return int(_load().swa_set_wait_timeout_ns(int(ns)))
+
+
+def swa_set_debug_flags(flags: int) -> int:
+    return _load().swa_set_debug_flags(int(flags))

@@ -1,0 +1,63 @@
+// Internal launch interfaces shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace swa {
+
+constexpr int kBM = 128;            // query rows per prefill tile (TMEM lanes)
+constexpr int kBN = 128;            // keys per prefill tile
+constexpr int kMaxSeqSmem = 1024;   // varlen sequences whose tables fit in shared memory
+
+struct PrefillArgs {
+  void* out;
+  float* lse;                 // may be null
+  const int32_t* cu_seqlens;  // null: n_seq sequences of length L laid end to end
+  int n_seq;
+  int L;
+  long long T;                // total tokens
+  int Hq, Hkv, G;
+  int window, n_sink;
+  float scale;
+  float scale_log2;           // scale * log2(e)
+  int lse_varlen;             // 1: lse [Hq, T]; 0: lse [n_seq, Hq, L]
+  int total_tiles;            // fixed length: n_seq * ceil(L / kBM); varlen: computed on device
+  unsigned long long timeout_ns;
+  int debug_flags;
+  int* err;
+};
+
+// Launch the persistent prefill kernel (d = 64 or 128; bf16 in with bf16 or fp32 out, or
+// fp32 in and out with d = 64).
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tv, int d, bool f32, bool out_f32, int grid,
+                           cudaStream_t stream);
+
+struct DecodeArgs {
+  const void* q;        // [B, Hq, d]
+  const void* kcache;   // [B, Hkv, W, d]
+  const void* vcache;
+  const void* sink_k;   // [B, Hkv, S, d]
+  const void* sink_v;
+  const int32_t* pos;   // [B]
+  void* out;            // [B, Hq, d]
+  float* lse;           // [B, Hq] or null
+  float* part;          // partial states, (n_warps + B*Hkv) slots
+  int B, Hq, Hkv, G, W, S;
+  float scale_log2;
+  int n_warps;          // total warps of the split kernel
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream);
+size_t decode_partial_floats(int G, int d);
+cudaError_t decode_occupancy(int d, int B, int* ctas_per_sm);
+int decode_threads();
+
+cudaError_t launch_cache_fill(const void* k, const void* v, int P, void* kc, void* vc, void* sk,
+                              void* sv, int B, int Hkv, int d, int W, int S, cudaStream_t stream);
+cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* pos, void* kc,
+                                void* vc, void* sk, void* sv, int B, int Hkv, int d, int W, int S,
+                                cudaStream_t stream);
+
+}  // namespace swa

@@ -1,0 +1,70 @@
+"""The C-ABI library loads and exports what include/swa.h declares (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sink_aware_sliding_b200 as swa
+from sink_aware_sliding_b200 import build as swa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "swa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    swa_build.build()
+    return swa.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(swa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(swa.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        ctypes.cast(getattr(lib, name), ctypes.c_void_p)
+
+
+def test_status_strings(lib):
+    assert swa.swa_status_string(0) == "ok"
+    assert "invalid" in swa.swa_status_string(1)
+    assert "timed out" in swa.swa_status_string(4)
+    assert swa.swa_status_string(99) == "unknown status"
+    assert swa.swa_version() == 0x000100
+
+
+def _fwd(lib, **kw):
+    args = dict(q=None, k=None, v=None, out=None, lse=None, B=1, Hq=4, Hkv=2, L=16, d=128,
+                window=8, n_sink=4, scale=0.1, dtype=0, stream=None)
+    args.update(kw)
+    return lib.swa_fwd(args["q"], args["k"], args["v"], args["out"], args["lse"], args["B"],
+                       args["Hq"], args["Hkv"], args["L"], args["d"], args["window"],
+                       args["n_sink"], ctypes.c_float(args["scale"]), args["dtype"], args["stream"])
+
+
+def test_argument_checks_happen_before_any_device_work(lib):
+    # These all return from host-side validation without touching CUDA.
+    assert _fwd(lib, Hq=3, Hkv=2) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, window=0) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, n_sink=-1) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf")) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=7) == swa.SWA_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == swa.SWA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=128, dtype=1) == swa.SWA_ERR_UNSUPPORTED
+    assert _fwd(lib, B=0) == swa.SWA_OK                     # empty: nothing to launch
+    assert _fwd(lib, L=0) == swa.SWA_OK
+    assert _fwd(lib) == swa.SWA_ERR_INVALID_ARG             # null pointers
+    assert _fwd(lib, q=16, k=32, v=48, out=64 + 8) == swa.SWA_ERR_INVALID_ARG  # misaligned
+    assert lib.swa_decode_workspace_bytes(1, 12, 1, 128, 64, 4) == 0    # G = 12 > 8
+    assert lib.swa_decode_workspace_bytes(1, 4, 3, 128, 64, 4) == 0     # Hq % Hkv != 0
+    assert lib.swa_decode_workspace_bytes(1, 4, 1, 80, 64, 4) == 0      # d = 80
