@@ -1,0 +1,625 @@
+#!/usr/bin/env python
+"""Benchmark of sink-aware sliding-window attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl swa|reference]
+                    [--workloads based_local,gqa8b_prefill,packed_long,decode]
+
+Prints ONE JSON line on rank 0.  The headline (`value`) is the prefill
+throughput in TFLOP/s of the Based-style local-window workload (B=8, H=16,
+L=2048, d=64, window 128), counting 4*d FLOPs per visible (query, key) pair.
+The same line carries, under "workloads", the other workloads measured the
+same way: the 8B-shaped GQA prefill and the packed long-context prefill
+(TFLOP/s against the tensor roofline) and the ring-buffer decode (HBM GB/s and
+tokens/s against the HBM roofline).
+
+Timing: inputs are generated on the device and stay resident; W untimed
+warm-up steps; K timed steps between a barrier plus device synchronisation on
+both sides; each prefill step is timed with CUDA events on the launching
+stream, with a 512 MiB buffer written between steps so L2 (126 MB) holds
+nothing of the next step's inputs; the decode cache (1.07 GB) is larger than
+L2 by itself.  Multi-GPU runs are replicas (weak scaling): every rank runs the
+same workload on its own GPU, times are reduced with a max over ranks.
+
+`e2e` is the same metric through the C ABI with the inputs in pinned host
+memory: each step copies its inputs host->device, runs the kernel(s) and
+copies the outputs back, all inside the timed region.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (the
+reference arm); it runs on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sink-SWA prefill TFLOP/s (visible pairs) & decode HBM GB/s, % of B200 roofline"
+HEADLINE = "based_local"
+L2_FLUSH_BYTES = 512 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- counting
+def visible_pairs(L: int, w: int, s: int) -> int:
+    """Sum over query rows t < L of the number of visible keys min(t+1, w) + clamp(t-w+1, 0, s)."""
+    if L <= 0:
+        return 0
+    band = L * (L + 1) // 2 if L <= w else w * (w + 1) // 2 + (L - w) * w
+    n = L - w                      # rows whose window starts past position 0
+    if n <= 0:
+        sinks = 0
+    elif n <= s:
+        sinks = n * (n + 1) // 2
+    else:
+        sinks = s * (s + 1) // 2 + (n - s) * s
+    return band + sinks
+
+
+def prefill_flops(w, seqlens) -> int:
+    return 4 * w.d * w.Hq * sum(visible_pairs(n, w.window, w.n_sink) for n in seqlens)
+
+
+def prefill_bytes(w, T: int, in_bytes: int = 2, out_bytes: int = 2) -> int:
+    return T * (w.Hq + 2 * w.Hkv) * w.d * in_bytes + T * w.Hq * w.d * out_bytes + T * w.Hq * 4
+
+
+def decode_step_bytes(w, pos: int) -> int:
+    keys = min(pos + 1, w.window) + min(max(pos - w.window + 1, 0), w.n_sink)
+    cache = w.B * w.Hkv * keys * w.d * 2 * 2
+    qo = 2 * w.B * w.Hq * w.d * 2 + w.B * w.Hq * 4
+    append = 2 * (2 * w.B * w.Hkv * w.d * 2)     # read k_new, v_new and write them
+    return cache + qo + append
+
+
+def decode_step_flops(w, pos: int) -> int:
+    keys = min(pos + 1, w.window) + min(max(pos - w.window + 1, 0), w.n_sink)
+    return 4 * w.d * w.B * w.Hq * keys
+
+
+# --------------------------------------------------------------------------- distributed
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while active (read only)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            h = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = None
+            if h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_device.index]) if vis and vis.split(",")[0].isdigit() \
+                    else torch_device.index
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _reasons_now(self):
+        nv = self._nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                try:
+                    return getattr(nv, fn)(self._h)
+                except Exception:
+                    pass
+        return 0
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = self._reasons_now()
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._stop.clear()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            self._thread = None
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(PEAKS_FALLBACK, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sink_aware_sliding_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the workload's dominant kernel from the committed ncu
+    summary, or None if the kernels changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class Timer:
+    """CUDA events around single launches on the current stream."""
+
+    def __init__(self, torch):
+        self.torch = torch
+        self.pairs = []
+
+    def __call__(self, fn):
+        t = self.torch
+        e0, e1 = t.cuda.Event(enable_timing=True), t.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        self.pairs.append((e0, e1))
+
+    def ms(self):
+        self.torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in self.pairs]
+
+
+# --------------------------------------------------------------------------- workloads (GPU)
+def bench_prefill(name, steps, warmup, dev, flush, peaks, sampler):
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    varlen = w.kind == "varlen"
+    if varlen:
+        q, k, v, cu = wl.make_varlen(w, device=dev)
+        seqlens, T = list(w.seqlens), cu[-1]
+        cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
+        lse = torch.empty(w.Hq, T, device=dev, dtype=torch.float32)
+    else:
+        q, k, v = wl.make_prefill(w, device=dev)
+        seqlens, T = [w.L] * w.B, w.B * w.L
+        lse = torch.empty(w.B, w.Hq, w.L, device=dev, dtype=torch.float32)
+    out = torch.empty_like(q)
+
+    def run(qq=q, kk=k, vv=v, oo=out, ll=lse):
+        if varlen:
+            swa.swa_fwd_varlen(qq, kk, vv, oo, ll, cu_d, w.window, w.n_sink)
+        else:
+            swa.swa_fwd(qq, kk, vv, oo, ll, w.window, w.n_sink)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    if swa.swa_device_error() != 0:
+        raise RuntimeError(f"{name}: device wait timed out")
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)             # evict the previous step's data from L2 (untimed)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    per = timer.ms()
+    ms = reduce_max(sum(per), dev) / steps
+    flops = prefill_flops(w, seqlens)
+    alg_bytes = prefill_bytes(w, T)
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    hbm_bound = flops / alg_bytes < peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+
+    # end to end through the C ABI with pinned host buffers
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        run(dq, dk, dv, out, lse)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, steps // 2)
+    barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    if hbm_bound:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"]}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                "peak_source": peaks["source"]}
+    roof["traffic"] = profiled_traffic(name)
+    roof["algorithmic_bytes_per_launch"] = alg_bytes
+    roof["flops_per_launch"] = flops
+    return {
+        "config": w.describe(), "value": round(tflops, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+        "achieved_gbs": round(gbs, 1), "roofline": roof,
+        "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
+def bench_decode(name, steps, warmup, dev, peaks, sampler):
+    """One step = one generated token for all B sequences: cache append + split-K decode + merge."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    n_tok = steps                      # generated tokens timed
+    di = wl.make_decode(w, device=dev, steps=n_tok + warmup)
+    B, Hq, Hkv, d, W, S = w.B, w.Hq, w.Hkv, w.d, w.window, w.n_sink
+    z = dict(device=dev, dtype=torch.bfloat16)
+    kc, vc = torch.empty(B, Hkv, W, d, **z), torch.empty(B, Hkv, W, d, **z)
+    sk, sv = torch.empty(B, Hkv, S, d, **z), torch.empty(B, Hkv, S, d, **z)
+    swa.swa_cache_fill(di.prefix_k, di.prefix_v, kc, vc, sk, sv, W, S)
+    del di.prefix_k, di.prefix_v
+    pos = torch.arange(w.prefix, w.prefix + n_tok + warmup, dtype=torch.int32, device=dev)
+    pos = pos.view(-1, 1).expand(-1, B).contiguous()
+    out = torch.empty(B, Hq, d, **z)
+    lse = torch.empty(B, Hq, device=dev, dtype=torch.float32)
+    ws = torch.empty(swa.swa_decode_workspace_bytes(B, Hq, Hkv, d, W, S), device=dev, dtype=torch.uint8)
+
+    def step(i):
+        swa.swa_cache_append(di.k_new[i], di.v_new[i], pos[i], kc, vc, sk, sv, W, S)
+        swa.swa_decode(di.q[i], kc, vc, sk, sv, pos[i], out, lse, W, S, ws)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        e0.record()
+        for i in range(warmup, warmup + n_tok):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(e0.elapsed_time(e1), dev) / n_tok
+    # dominant kernel (split-K decode + merge) timed per call on the same stream
+    timer = Timer(torch)
+    for i in range(warmup, warmup + min(n_tok, 64)):
+        timer(lambda i=i: swa.swa_decode(di.q[i], kc, vc, sk, sv, pos[i], out, lse, W, S, ws))
+    dec_ms = statistics.mean(timer.ms())
+    p_last = w.prefix + warmup + n_tok - 1
+    step_bytes = decode_step_bytes(w, p_last)
+    dec_bytes = step_bytes - 2 * (2 * B * Hkv * d * 2)      # the decode call alone
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    tok_s = B / (ms * 1e-3)
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    # end to end: per step copy q, k_new, v_new, pos host->device and out, lse back
+    hq, hk, hv = di.q[0].cpu().pin_memory(), di.k_new[0].cpu().pin_memory(), di.v_new[0].cpu().pin_memory()
+    hp = pos[warmup].cpu().pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv, dp = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hp))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dp.copy_(hp, non_blocking=True)
+        swa.swa_cache_append(dk, dv, dp, kc, vc, sk, sv, W, S)
+        swa.swa_decode(dq, kc, vc, sk, sv, dp, out, lse, W, S, ws)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(8, n_tok // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hp))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    return {
+        "config": w.describe(), "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
+        "tokens_per_s": round(tok_s, 1), "tflops": round(decode_step_flops(w, p_last) / (ms * 1e-3) / 1e12, 2),
+        "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(dec_gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+                     "traffic": profiled_traffic(name), "algorithmic_bytes_per_launch": dec_bytes,
+                     "kernel_ms": round(dec_ms, 5), "step_frac": round(gbs / peaks["hbm_gbs"], 4)},
+        "e2e": {"value": round(B / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * n_tok, "l2": "cache of 1.07 GB exceeds L2",
+    }
+
+
+# --------------------------------------------------------------------------- oracle (CPU)
+def oracle_rate(name: str, min_seconds: float = 10.0, max_seconds: float = 30.0):
+    """The fp64 oracle on the host cores over a bounded sample of the workload.
+    Returns (TFLOP/s, cores, sample description)."""
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    cores = oracle.num_threads()
+    if w.kind == "prefill" and w.B * w.L * w.Hq <= 8 * 2048 * 16:
+        q, k, v = wl.make_prefill(w)
+        flops = prefill_flops(w, [w.L] * w.B)
+        sample = f"whole workload ({w.B} sequences x {w.L} rows x {w.Hq} heads), repeated"
+        passes, t0 = 0, time.perf_counter()
+        while True:
+            oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
+            passes += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_seconds or dt * (passes + 1) / passes > max_seconds:
+                break
+        return flops * passes / dt / 1e12, cores, f"{sample} {passes} times in {dt:.1f} s"
+    raise ValueError(f"no CPU sample defined for {name}")
+
+
+def reference_arm(args):
+    """The fp64 oracle as the reference arm: each step is one pass over a bounded sample."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[HEADLINE]
+    q, k, v = wl.make_prefill(w, B=1)
+    flops = prefill_flops(w, [w.L])
+    cores = oracle.num_threads()
+    for _ in range(args.warmup):
+        oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
+    dt = time.perf_counter() - t0
+    val = flops * args.steps / dt / 1e12
+    sample = f"1 of {w.B} sequences ({w.L} rows x {w.Hq} heads) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded inputs)",
+        "config": dict(wl.WORKLOADS[HEADLINE].describe(), parallelism="host cores"),
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def profile_case(args):
+    """Launch one workload's kernels a few times at an optional smaller size (for ncu)."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.profile_case]
+    n = args.warmup + args.steps
+    if w.kind == "prefill":
+        q, k, v = wl.make_prefill(w, device=dev, B=args.B, L=args.L)
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[0], w.Hq, q.shape[1], device=dev, dtype=torch.float32)
+        for _ in range(n):
+            swa.swa_fwd(q, k, v, out, lse, w.window, w.n_sink)
+    elif w.kind == "varlen":
+        q, k, v, cu = wl.make_varlen(w, device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(w.Hq, cu[-1], device=dev, dtype=torch.float32)
+        cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
+        for _ in range(n):
+            swa.swa_fwd_varlen(q, k, v, out, lse, cu_d, w.window, w.n_sink)
+    else:
+        B = args.B or w.B
+        di = wl.make_decode(w, device=dev, B=B, steps=n)
+        z = dict(device=dev, dtype=torch.bfloat16)
+        kc, vc = torch.empty(B, w.Hkv, w.window, w.d, **z), torch.empty(B, w.Hkv, w.window, w.d, **z)
+        sk, sv = torch.empty(B, w.Hkv, w.n_sink, w.d, **z), torch.empty(B, w.Hkv, w.n_sink, w.d, **z)
+        swa.swa_cache_fill(di.prefix_k, di.prefix_v, kc, vc, sk, sv, w.window, w.n_sink)
+        out = torch.empty(B, w.Hq, w.d, **z)
+        lse = torch.empty(B, w.Hq, device=dev, dtype=torch.float32)
+        ws = torch.empty(swa.swa_decode_workspace_bytes(B, w.Hq, w.Hkv, w.d, w.window, w.n_sink),
+                         device=dev, dtype=torch.uint8)
+        for i in range(n):
+            pos = torch.full((B,), w.prefix + i, dtype=torch.int32, device=dev)
+            swa.swa_cache_append(di.k_new[i], di.v_new[i], pos, kc, vc, sk, sv, w.window, w.n_sink)
+            swa.swa_decode(di.q[i], kc, vc, sk, sv, pos, out, lse, w.window, w.n_sink, ws)
+    torch.cuda.synchronize()
+    if swa.swa_device_error() != 0:
+        raise SystemExit("device wait timed out")
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
+    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode")
+    ap.add_argument("--decode-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None,
+                    help="only launch this workload's kernels --warmup + --steps times and print "
+                         "nothing (a small, self-contained case for ncu captures)")
+    ap.add_argument("--L", type=int, default=None, help="with --profile-case: sequence length")
+    ap.add_argument("--B", type=int, default=None, help="with --profile-case: batch")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    if args.profile_case:
+        profile_case(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import datetime
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import sink_aware_sliding_b200 as swa
+    swa.library()
+
+    # CPU baseline first, before any large device allocation (rank 0, one GPU only).
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, cores, sample = oracle_rate(HEADLINE)
+        cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    peaks = load_peaks()
+    sampler = ClockSampler(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    names = [n for n in args.workloads.split(",") if n]
+    if HEADLINE not in names:
+        names.insert(0, HEADLINE)
+    results = {}
+    for n in names:
+        if n == "decode":
+            results[n] = bench_decode(n, args.decode_tokens, args.warmup, dev, peaks, sampler)
+        else:
+            results[n] = bench_prefill(n, args.steps, args.warmup, dev, flush, peaks, sampler)
+        torch.cuda.empty_cache()
+
+    head = results[HEADLINE]
+    clocks = sampler.summary()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    scale = world       # weak scaling: every rank ran the same work
+    line = {
+        "metric": METRIC,
+        "value": round(head["value"] * scale, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16; see workloads/__init__.py)",
+        "config": dict(head["config"], parallelism=f"replicas x{world}", l2=head["l2"]),
+        "roofline": head["roofline"],
+        "cpu_baseline": cpu,
+        "e2e": dict(head["e2e"], value=round(head["e2e"]["value"] * scale, 3)),
+        "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
+        "clocks": clocks,
+        "workloads": {n: r for n, r in results.items() if n != HEADLINE},
+        "kernel_hash": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
