@@ -136,6 +136,35 @@ int swa_decode(const void* q, const void* kcache, const void* vcache,
                int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
                void* workspace, size_t workspace_bytes, swa_stream_t stream);
 
+/*
+ * swa_decode without a workspace argument, for callers that cannot allocate
+ * device memory: code that runs inside a host framework which owns every
+ * device allocation (a serving engine with a preallocated arena, a plugin in
+ * somebody else's process), or under a rule that forbids cudaMalloc after
+ * start-up because allocation can stall the device or fail at the worst time.
+ * The pages have no counterpart; this is a packaging variant of swa_decode.
+ *
+ * Same arguments, layouts and results as swa_decode minus workspace and
+ * workspace_bytes.  The scratch for the partial softmax states is a fixed
+ * 8 MiB array compiled into the library (every GPU that loads the library
+ * holds it until the process exits); nothing is allocated, by the library or
+ * any library it calls.  Sizes whose scratch (swa_decode_workspace_bytes)
+ * exceeds 8 MiB are rejected with SWA_ERR_UNSUPPORTED and nothing is launched;
+ * for the 64 x 32 x 8 x 128 decode workload the need is about 3.5 MiB.
+ * The first call on each device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.  All calls on a device share the one array and
+ * it keeps whatever the last call left there; every value a call reads was
+ * written earlier in the same call, so nothing needs clearing, but calls
+ * whose work overlaps on the GPU (different streams, or different host
+ * threads) race on the array and must be serialised by the caller.
+ */
+int swa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                       const void* sink_k, const void* sink_v, const int32_t* pos,
+                       void* out, float* lse,
+                       int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
+                       swa_stream_t stream);
+
 /* Static text for a status code. */
 const char* swa_status_string(int status);
 

@@ -35,7 +35,7 @@ SWA_DTYPE_BF16_F32OUT = 2
 EXPORTS = (
     "swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append",
     "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
-    "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version",
+    "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
 )
 
 _lib = None
@@ -62,6 +62,7 @@ def _load():
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = SZ
     lib.swa_decode.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
@@ -69,6 +70,7 @@ def _load():
     lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
+                 "swa_decode_noalloc",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -187,6 +189,20 @@ def swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_
                             _scale(scale, d), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream))
     _check(st, "swa_decode")
+
+
+def swa_decode_noalloc(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,
+                       scale=None, stream=None) -> None:
+    """swa_decode for callers that cannot allocate device memory: the split-K
+    scratch lives in a fixed 8 MiB array inside the library instead of a
+    caller-provided workspace.  Calls that overlap on the GPU share that array
+    and must not run concurrently; sizes needing more than 8 MiB raise."""
+    B, Hq, d = q.shape
+    Hkv = kcache.shape[1]
+    st = _load().swa_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(sink_k), _ptr(sink_v),
+                                    _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window),
+                                    int(n_sink), _scale(scale, d), _stream(stream))
+    _check(st, "swa_decode_noalloc")
 
 
 def swa_device_error(stream=None) -> int:
