@@ -183,9 +183,11 @@ int swa_device_error(swa_stream_t stream);
 unsigned long long swa_set_wait_timeout_ns(unsigned long long ns);
 
 /*
- * Test hook, process-wide: flags = 1 makes the prefill kernel's load warp
- * issue no copies, so that its consumers' bounded waits run out.  0 restores
- * normal operation.  Returns the previous flags.
+ * Test hooks, process-wide.  Bit 0 makes the prefill kernels' load warp issue
+ * no copies, so that its consumers' bounded waits run out; bit 1 makes
+ * swa_fwd / swa_fwd_varlen use the one-query-tile kernel even where the
+ * two-tile kernel applies.  0 restores normal operation.  Returns the
+ * previous flags.
  */
 int swa_set_debug_flags(int flags);
 

@@ -1,0 +1,269 @@
+// Pieces shared by the prefill kernels: work-unit decoding (which key tiles a
+// query tile visits), bounded barrier waits, the per-tile online softmax on a
+// row held in tensor memory, and the epilogue that writes O and LSE.
+//
+// Visible set ("Sliding-window beats linear attention", sections 1 and 3):
+// row t sees key j iff j <= t and (j >= t - window + 1 or j < n_sink).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "swa_internal.h"
+
+namespace swa {
+namespace prefill {
+
+constexpr int kStatusTimeout = 4;  // SWA_ERR_DEVICE_TIMEOUT
+
+// One query tile of one head: rows [m0, m1] of sequence seq, and its key tiles:
+// first the nst tiles of the sink prefix that lie left of the band, then the
+// band tiles kb_lo .. kb_lo + n_tiles - nst - 1.
+struct Unit {
+  int seq, seq_start, len, m0, m1, nst, kb_lo, n_tiles;
+};
+
+struct Ctl {
+  volatile int* abort_flag;
+  const PrefillArgs* a;
+};
+
+__device__ __forceinline__ void fail(const Ctl& c) {
+  *c.abort_flag = 1;
+  atomicCAS(c.a->err, 0, kStatusTimeout);
+}
+
+// Bounded wait on (bar, parity).  False if the time limit ran out (which starts
+// the CTA's abort) or, when honor_abort is set, as soon as another thread has
+// started it.  Teardown waits pass honor_abort = false.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl c, bool honor_abort = true) {
+  for (int i = 0; i < 256; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (honor_abort && *c.abort_flag) return false;
+    if (globaltimer_ns() - t0 > c.a->timeout_ns) {
+      fail(c);
+      return false;
+    }
+  }
+}
+
+// Query tile number gt (0 = first tile of the first sequence) -> unit geometry.
+// Varlen sequences are found in the shared tables: s_cu (cu_seqlens copy) and
+// s_tpre (query tiles before each sequence).
+__device__ __forceinline__ void decode_tile(const PrefillArgs& a, const int* s_cu, const int* s_tpre,
+                                            int gt, Unit& x) {
+  int qt;
+  if (a.cu_seqlens == nullptr) {
+    const int tps = (a.L + kBM - 1) / kBM;
+    x.seq = gt / tps;
+    qt = gt - x.seq * tps;
+    x.seq_start = x.seq * a.L;
+    x.len = a.L;
+  } else {
+    int lo = 0, hi = a.n_seq - 1;  // last sequence with s_tpre[seq] <= gt (skips empty ones)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tpre[mid] <= gt) lo = mid; else hi = mid - 1;
+    }
+    x.seq = lo;
+    qt = gt - s_tpre[lo];
+    x.seq_start = s_cu[lo];
+    x.len = s_cu[lo + 1] - s_cu[lo];
+  }
+  x.m0 = qt * kBM;
+  x.m1 = min(x.m0 + kBM, x.len) - 1;
+  const int lo_key = max(0, x.m0 - a.window + 1);
+  x.kb_lo = lo_key / kBN;
+  const int kb_hi = x.m1 / kBN;
+  x.nst = a.n_sink > 0 ? min((a.n_sink + kBN - 1) / kBN, x.kb_lo) : 0;
+  x.n_tiles = x.nst + kb_hi - x.kb_lo + 1;
+}
+
+__device__ __forceinline__ int tile_n0(const Unit& x, int j) {
+  return (j < x.nst ? j : x.kb_lo + (j - x.nst)) * kBN;
+}
+
+// Does key tile j of unit x hold any key some row of the tile cannot see?
+__device__ __forceinline__ bool tile_needs_mask(const Unit& x, int j, int window) {
+  const int n0 = tile_n0(x, j);
+  return (j < x.nst) || (n0 + kBN - 1 > x.m0) || (n0 < x.m1 - window + 1);
+}
+
+// Warp 0 builds the varlen tables (cu_seqlens copy and query-tile prefix sums).
+__device__ __forceinline__ void build_varlen_tables(const PrefillArgs& a, int* s_cu, int* s_tpre,
+                                                    int lane) {
+  const int n = a.n_seq;
+  const int per = (n + 31) / 32;
+  int local = 0;
+  for (int i = lane * per; i < min(n, (lane + 1) * per); ++i) {
+    const int c0 = a.cu_seqlens[i], c1 = a.cu_seqlens[i + 1];
+    s_cu[i] = c0;
+    local += (c1 - c0 + kBM - 1) / kBM;
+  }
+  if (lane == 0) s_cu[n] = a.cu_seqlens[n];
+  int incl = local;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  int run = incl - local;
+  for (int i = lane * per; i < min(n, (lane + 1) * per); ++i) {
+    s_tpre[i] = run;
+    run += (a.cu_seqlens[i + 1] - a.cu_seqlens[i] + kBM - 1) / kBM;
+  }
+  if (lane == 31) s_tpre[n] = incl;
+}
+
+// Online softmax of one key tile for the row this thread owns (TMEM lane).
+// Reads S from s_tmem (128 fp32 columns), masks it if the tile needs it,
+// moves the reference max only when it grew by more than 2^8 in exp2 units,
+// writes P over S (packed bf16 pairs, or fp32 for the tf32 path) and updates
+// the running max and sum.  Returns whether the reference max moved; alpha is
+// the factor the row's O accumulator must be scaled by in that case.
+template <bool F32>
+__device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, const Unit& x, int j, int t,
+                                             const PrefillArgs& a, float& m_run, float& l_run,
+                                             float& alpha) {
+  const float sl2 = a.scale_log2;
+  float s[kBN];
+  {
+    uint32_t sr[kBN];
+    tmem_ld128_wait(s_tmem, sr);
+#pragma unroll
+    for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(sr[i]);
+  }
+  if (tile_needs_mask(x, j, a.window)) {
+    const int n0 = tile_n0(x, j);
+    const int hi = t - n0;                 // visible: c <= hi
+    const int lo = t - a.window + 1 - n0;  //   and (c >= lo
+    const int sk = a.n_sink - n0;          //        or c < sk)
+#pragma unroll
+    for (int c = 0; c < kBN; ++c) {
+      const bool vis = (c <= hi) && (c >= lo || c < sk);
+      s[c] = vis ? s[c] : -INFINITY;
+    }
+  }
+  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+  for (int c = 4; c < kBN; c += 4) {
+    mx0 = fmaxf(mx0, s[c]);
+    mx1 = fmaxf(mx1, s[c + 1]);
+    mx2 = fmaxf(mx2, s[c + 2]);
+    mx3 = fmaxf(mx3, s[c + 3]);
+  }
+  const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+  const float m_new = fmaxf(m_run, mx);
+  // NaN from (-inf) - (-inf) compares false: a row with nothing visible yet keeps -inf.
+  const bool need = (m_new - m_run) * sl2 > 8.0f;
+  const float m_use = need ? m_new : m_run;
+  alpha = need ? ex2_approx((m_run - m_new) * sl2) : 1.0f;
+  const float neg = (m_use == -INFINITY) ? 0.0f : -m_use * sl2;
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < kBN; c += 2) {
+    s[c] = ex2_approx(fmaf(s[c], sl2, neg));
+    s[c + 1] = ex2_approx(fmaf(s[c + 1], sl2, neg));
+    sum0 += s[c];
+    sum1 += s[c + 1];
+  }
+  l_run = l_run * alpha + (sum0 + sum1);
+  m_run = m_use;
+  if constexpr (F32) {
+#pragma unroll
+    for (int c = 0; c < kBN / 32; ++c) {
+      uint32_t pr[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pr[i] = __float_as_uint(s[c * 32 + i]);
+      tmem_st32(s_tmem + c * 32, pr);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < kBN / 64; ++c) {
+      uint32_t pr[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pr[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
+      tmem_st32(s_tmem + c * 32, pr);
+    }
+  }
+  return need;
+}
+
+// Scale this warp's 32 rows of O (d columns at o_tmem) by alpha (per row).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t rr[32];
+    tmem_ld32_wait(o_tmem + c * 32, rr);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+    tmem_st32(o_tmem + c * 32, rr);
+  }
+}
+
+// O / l of this thread's row (d columns at o_tmem) -> out, and the row's LSE.
+template <int D, bool OUT_F32>
+__device__ __forceinline__ void store_row(uint32_t o_tmem, const PrefillArgs& a, const Unit& x,
+                                          int h, int t, float m_run, float l_run) {
+  const bool valid = t < x.len;
+  const float inv_l = 1.0f / l_run;
+  const size_t row = static_cast<size_t>(x.seq_start) + static_cast<size_t>(t);
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t rr[32];
+    tmem_ld32_wait(o_tmem + c * 32, rr);
+    if (!valid) continue;
+    if constexpr (OUT_F32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (row * a.Hq + h) * D + c * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_float4(__uint_as_float(rr[4 * i]) * inv_l, __uint_as_float(rr[4 * i + 1]) * inv_l,
+                             __uint_as_float(rr[4 * i + 2]) * inv_l, __uint_as_float(rr[4 * i + 3]) * inv_l);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (row * a.Hq + h) * D + c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(rr[8 * i + 0]) * inv_l, __uint_as_float(rr[8 * i + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(rr[8 * i + 2]) * inv_l, __uint_as_float(rr[8 * i + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(rr[8 * i + 4]) * inv_l, __uint_as_float(rr[8 * i + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(rr[8 * i + 6]) * inv_l, __uint_as_float(rr[8 * i + 7]) * inv_l);
+        dst[i] = w;
+      }
+    }
+  }
+  if (valid && a.lse != nullptr) {
+    const float ref = (m_run == -INFINITY) ? 0.0f : m_run * a.scale_log2;
+    const float lse = (ref + log2f(l_run)) * 0.69314718055994531f;
+    const size_t idx = a.lse_varlen ? static_cast<size_t>(h) * static_cast<size_t>(a.T) + row
+                                    : (static_cast<size_t>(x.seq) * a.Hq + h) * a.L + t;
+    a.lse[idx] = lse;
+  }
+}
+
+// Shared-memory matrix descriptors of the operands (see the kernels for the layouts).
+// K-major tile of `rows` rows x (NCHUNK x 128 bytes), 128-byte swizzle: MMA k-step kk of
+// 32 bytes lies in column chunk kk / steps_per_chunk.
+template <int STEPS_PER_CHUNK>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int rows, int kk) {
+  const int ch = kk / STEPS_PER_CHUNK;
+  const int wi = kk % STEPS_PER_CHUNK;
+  return smem_desc(tile_base + ch * (rows * 128) + wi * 32, 16, 1024, kLayoutSw128);
+}
+// V as the MN-major B operand of O += P V: k-step kk covers KSTEP key rows; LBO jumps
+// between 128-byte column chunks of d (kBN rows apart); SBO between swizzle atoms along
+// the keys (8 rows; tf32 operands in MN-major order need the 32-byte-atom swizzle whose
+// atom is 4 rows).
+template <bool F32, int KSTEP>
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile_base, int kk) {
+  return F32 ? smem_desc(tile_base + kk * (KSTEP * 128), kBN * 128, 512, kLayoutSw128Atom32)
+             : smem_desc(tile_base + kk * (KSTEP * 128), kBN * 128, 1024, kLayoutSw128);
+}
+
+}  // namespace prefill
+}  // namespace swa

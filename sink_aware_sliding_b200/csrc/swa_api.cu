@@ -136,9 +136,17 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
     units = (T / swa::kBM + n_seq) * static_cast<long long>(Hq);  // upper bound
     if (units > INT32_MAX) return SWA_ERR_UNSUPPORTED;
   }
+  // Debug flag 2 forces the one-tile kernel (so tests can check both kernels).
+  const bool pair = (a.debug_flags & 2) == 0 && swa::prefill_pair_supported(Hq, Hq / Hkv, d, f32);
+  if (pair) units = (units + 1) / 2;
   const int grid = static_cast<int>(std::min<long long>(dev->sms, units));
   if (grid <= 0) return SWA_OK;
-  cudaError_t e = swa::launch_prefill(a, tq, tk, tv, d, f32, dtype != SWA_DTYPE_BF16, grid, stream);
+  cudaError_t e = cudaErrorNotSupported;
+  if (pair) e = swa::launch_prefill_pair(a, tq, tk, tv, d, f32, dtype != SWA_DTYPE_BF16, grid, stream);
+  if (e == cudaErrorNotSupported) {  // one-tile kernel (odd Hq, or the two-tile kernel declined)
+    const int grid1 = static_cast<int>(std::min<long long>(dev->sms, pair ? 2 * units : units));
+    e = swa::launch_prefill(a, tq, tk, tv, d, f32, dtype != SWA_DTYPE_BF16, grid1, stream);
+  }
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

@@ -34,6 +34,13 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
                            const CUtensorMap& tv, int d, bool f32, bool out_f32, int grid,
                            cudaStream_t stream);
 
+// Two-query-tile prefill (heads 2p, 2p+1 per CTA); used when Hq is even and the
+// ring can hold two key tiles (always for 16 KB tiles, else when pairs share a KV head).
+bool prefill_pair_supported(int Hq, int G, int d, bool f32);
+cudaError_t launch_prefill_pair(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, int d, bool f32, bool out_f32, int grid,
+                                cudaStream_t stream);
+
 struct DecodeArgs {
   const void* q;        // [B, Hq, d]
   const void* kcache;   // [B, Hkv, W, d]

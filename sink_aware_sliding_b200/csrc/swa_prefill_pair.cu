@@ -1,0 +1,365 @@
+// Prefill, two query tiles per CTA (query heads 2p and 2p+1 of the same 128
+// rows), sm_100a.
+//
+// Work unit = (sequence, 128-row query tile, head pair).  Both tiles visit the
+// same key tiles (the band plus the sink prefix, nothing else); when the two
+// heads read the same KV head (grouped-query attention with an even group) the
+// K and V tiles are loaded once for both.
+//
+// Roles (384 threads):
+//   warps 0-3   softmax of tile A (thread r = query row r = TMEM lane r)
+//   warps 4-7   softmax of tile B
+//   warp 8      TMA: the two Q tiles of a unit, then per key tile its K and V
+//               tiles, each into the next slot of one ring of tile-sized slots
+//   warp 9      tcgen05.mma issue (one thread) and TMEM allocation
+// The MMA order per key tile j is
+//   O_A += P_A(j) V(j);  S_A = Q_A K(j+1)^T;  O_B += P_B(j) V(j);  S_B = Q_B K(j+1)^T
+// so the tensor pipe works on one tile's products while the softmax warps of the
+// other tile run.  Each tile has a single S region in TMEM (P overwrites S in
+// place); because the MMAs of one CTA execute in issue order, S_X(j+1) being
+// ready implies O_X += P_X(j) V(j) has finished, so a softmax warp may rescale
+// its O rows right after reading S without a further barrier.
+// TMEM columns: S_A 0-127, S_B 128-255, O_A 256.., O_B 256+D.. (512 allocated).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "prefill_common.cuh"
+
+namespace swa {
+namespace {
+
+using namespace prefill;
+
+constexpr int kPairThreads = 384;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+// Register split: launched at 168 per thread (65536 / 384 rounded down to 8) =
+// 64512 in all; the load/MMA warpgroup gives back 168 - 88 = 80 per thread
+// (10240) and the two softmax warpgroups take 208 - 168 = 40 per thread (10240):
+// 2 * 128 * 208 + 128 * 88 = 64512.  The host checks the launch count first.
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kProducerRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs == kPairThreads * kLaunchRegs,
+              "register split must use exactly the registers the block is launched with");
+
+template <int D, bool F32>
+struct PairCfg {
+  static constexpr int ELEM = F32 ? 4 : 2;
+  static constexpr int CHUNK = 128 / ELEM;          // elements per 128-byte swizzled row
+  static constexpr int NCHUNK = D / CHUNK;
+  static constexpr int KSTEP = 32 / ELEM;           // K of one MMA instruction (32 bytes)
+  static constexpr int QK_STEPS = D / KSTEP;
+  static constexpr int PV_STEPS = kBN / KSTEP;
+  static constexpr int TILE = kBM * D * ELEM;       // bytes of one Q, K or V tile
+  static constexpr int QBUF = TILE <= 16384 ? 2 : 1;     // Q pairs in flight across units
+  static constexpr int NSTAGE = TILE <= 16384 ? 8 : 4;   // ring slots, each one K or V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + QBUF * 2 * TILE;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * TILE;
+  // barrier indices
+  static constexpr int B_QFULL = 0, B_QEMPTY = QBUF, B_FULL = 2 * QBUF, B_EMPTY = B_FULL + NSTAGE,
+                       B_SFULL = B_EMPTY + NSTAGE, B_PFULL = B_SFULL + 2, B_OFINAL = B_PFULL + 2,
+                       B_DRAIN = B_OFINAL + 2, NBAR = B_DRAIN + 1;
+  static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
+  static constexpr int OFF_ABORT = OFF_TMEMPTR + 4;
+  static constexpr int OFF_TABLES = OFF_ABORT + 12;
+  static constexpr int SMEM_BYTES = OFF_TABLES + 2 * 4 * (kMaxSeqSmem + 1) + 1024;
+  static constexpr uint32_t IDESC_QK = make_idesc(F32 ? 2u : 1u, kBM, kBN, false);
+  static constexpr uint32_t IDESC_PV = make_idesc(F32 ? 2u : 1u, kBM, D, true);
+  __device__ static constexpr uint32_t tmem_s(int half) { return half ? 128u : 0u; }
+  __device__ static constexpr uint32_t tmem_o(int half) { return 256u + (half ? D : 0); }
+};
+
+template <int D, bool F32, bool OUT_F32>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    swa_prefill_pair_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
+                            const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+  using C = PairCfg<D, F32>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8 * i; };
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_ABORT);
+  int* s_cu = reinterpret_cast<int*>(gbase + C::OFF_TABLES);
+  int* s_tpre = s_cu + (kMaxSeqSmem + 1);
+  const Ctl ctl{abort_flag, &a};
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::QBUF; ++i) {
+      mbar_init(bar(C::B_QFULL + i), 1);
+      mbar_init(bar(C::B_QEMPTY + i), 1);
+    }
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(bar(C::B_FULL + i), 1);
+      mbar_init(bar(C::B_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_SFULL + i), 1);
+      mbar_init(bar(C::B_PFULL + i), 128);
+      mbar_init(bar(C::B_OFINAL + i), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  if (a.cu_seqlens != nullptr && warp == 0) build_varlen_tables(a, s_cu, s_tpre, lane);
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_ptr), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int total_tiles = a.cu_seqlens != nullptr ? s_tpre[a.n_seq] : a.total_tiles;
+  const uint32_t tmem = *tmem_ptr;
+  const int n_pairs = a.Hq / 2;
+  const int n_units = total_tiles * n_pairs;
+  // unit u -> (tile, head pair): heaviest (latest) tiles first
+  auto unit_of = [&](int u, Unit& x, int& hA) {
+    decode_tile(a, s_cu, s_tpre, total_tiles - 1 - u / n_pairs, x);
+    hA = 2 * (u % n_pairs);
+  };
+
+  if (warp >= 8) {
+  // The load/MMA warpgroup hands registers to the softmax warpgroups (all four of
+  // its warps execute this; warps 10 and 11 have no further work).
+  regs_dec<kProducerRegs>();
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const bool skip = (a.debug_flags & 1) != 0;
+      bool ok = !skip;
+      int ld = 0, uc = 0;
+      int last_fill[C::NSTAGE];
+      int last_q[C::QBUF];
+      for (int i = 0; i < C::NSTAGE; ++i) last_fill[i] = -1;
+      for (int i = 0; i < C::QBUF; ++i) last_q[i] = -1;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
+        Unit x;
+        int hA;
+        unit_of(u, x, hA);
+        const int kvA = hA / a.G, kvB = (hA + 1) / a.G;
+        const bool shared = kvA == kvB;
+        const int qb = uc % C::QBUF;
+        if (!(ok = wait_bar(bar(C::B_QEMPTY + qb), ((uc / C::QBUF) & 1) ^ 1, ctl))) break;
+        mbar_expect_tx(bar(C::B_QFULL + qb), 2 * C::TILE);
+        for (int half = 0; half < 2; ++half)
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_3d(base + C::OFF_Q + (qb * 2 + half) * C::TILE + c * (kBM * 128), &tq,
+                        bar(C::B_QFULL + qb), c * C::CHUNK, hA + half, x.seq_start + x.m0);
+        last_q[qb] = uc;
+        for (int j = 0; ok && j < x.n_tiles; ++j) {
+          const int row = x.seq_start + tile_n0(x, j);
+          // slots: K_A, [K_B], V_A, [V_B]
+          for (int part = 0; part < (shared ? 2 : 4); ++part, ++ld) {
+            const int st = ld % C::NSTAGE;
+            if (!(ok = wait_bar(bar(C::B_EMPTY + st), ((ld / C::NSTAGE) & 1) ^ 1, ctl))) break;
+            const bool is_v = shared ? part == 1 : part >= 2;
+            const int kvh = shared ? kvA : ((part & 1) ? kvB : kvA);
+            mbar_expect_tx(bar(C::B_FULL + st), C::TILE);
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_load_3d(base + C::OFF_RING + st * C::TILE + c * (kBN * 128), is_v ? &tv : &tk,
+                          bar(C::B_FULL + st), c * C::CHUNK, kvh, row);
+            last_fill[st] = ld;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // Let copies already in flight land before the CTA exits.
+        for (int st = 0; st < C::NSTAGE; ++st)
+          if (last_fill[st] >= 0) wait_bar(bar(C::B_FULL + st), (last_fill[st] / C::NSTAGE) & 1, ctl, false);
+        for (int qb = 0; qb < C::QBUF; ++qb)
+          if (last_q[qb] >= 0) wait_bar(bar(C::B_QFULL + qb), (last_q[qb] / C::QBUF) & 1, ctl, false);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int ld = 0, uc = 0, cnt = 0;  // ring counter, units, key tiles processed (both halves)
+      auto wait_full = [&](int slot_ctr) -> bool {
+        return wait_bar(bar(C::B_FULL + slot_ctr % C::NSTAGE), (slot_ctr / C::NSTAGE) & 1, ctl);
+      };
+      auto slot_addr = [&](int slot_ctr) -> uint32_t {
+        return base + C::OFF_RING + (slot_ctr % C::NSTAGE) * C::TILE;
+      };
+      auto qk = [&](int half, uint32_t q_tile, int k_ctr) {
+        const uint32_t k_tile = slot_addr(k_ctr);
+#pragma unroll
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<F32>(tmem + C::tmem_s(half), kmajor_desc<C::QK_STEPS / C::NCHUNK>(q_tile, kBM, kk),
+                       kmajor_desc<C::QK_STEPS / C::NCHUNK>(k_tile, kBN, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+        tc_commit(bar(C::B_SFULL + half));
+      };
+      auto pv = [&](int half, int v_ctr, bool first) {
+        const uint32_t v_tile = slot_addr(v_ctr);
+#pragma unroll
+        for (int kk = 0; kk < C::PV_STEPS; ++kk)
+          umma_ts<F32>(tmem + C::tmem_o(half), tmem + C::tmem_s(half) + kk * 8,
+                       v_desc<F32, C::KSTEP>(v_tile, kk), C::IDESC_PV, (first && kk == 0) ? 0u : 1u);
+      };
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
+        Unit x;
+        int hA;
+        unit_of(u, x, hA);
+        const bool shared = hA / a.G == (hA + 1) / a.G;
+        const int per = shared ? 2 : 4;
+        const int qb = uc % C::QBUF;
+        const uint32_t qA = base + C::OFF_Q + (qb * 2) * C::TILE, qB = qA + C::TILE;
+        if (!(ok = wait_bar(bar(C::B_QFULL + qb), (uc / C::QBUF) & 1, ctl))) break;
+        // slots of tile j: base b_j = ld + j*per; K_A = b_j, K_B = b_j + (shared ? 0 : 1),
+        // V_A = b_j + (shared ? 1 : 2), V_B = V_A + (shared ? 0 : 1)
+        auto kA = [&](int j) { return ld + j * per; };
+        auto kB = [&](int j) { return ld + j * per + (shared ? 0 : 1); };
+        auto vA = [&](int j) { return ld + j * per + (shared ? 1 : 2); };
+        auto vB = [&](int j) { return ld + j * per + (shared ? 1 : 3); };
+        // prologue: S_A(0), S_B(0)
+        if (!(ok = wait_full(kA(0)) && (shared || wait_full(kB(0))))) break;
+        tc_fence_after();
+        qk(0, qA, kA(0));
+        qk(1, qB, kB(0));
+        tc_commit(bar(C::B_EMPTY + kA(0) % C::NSTAGE));
+        if (!shared) tc_commit(bar(C::B_EMPTY + kB(0) % C::NSTAGE));
+        if (x.n_tiles == 1) tc_commit(bar(C::B_QEMPTY + qb));
+        for (int j = 0; j < x.n_tiles; ++j, ++cnt) {
+          const bool last = j == x.n_tiles - 1;
+          // ---- tile A: O_A += P_A(j) V(j), then S_A(j+1)
+          if (!(ok = wait_bar(bar(C::B_PFULL + 0), cnt & 1, ctl) && wait_full(vA(j)))) break;
+          tc_fence_after();
+          pv(0, vA(j), j == 0);
+          if (last) tc_commit(bar(C::B_OFINAL + 0));
+          if (!last) {
+            if (!(ok = wait_full(kA(j + 1)) && (shared || wait_full(kB(j + 1))))) break;
+            tc_fence_after();
+            qk(0, qA, kA(j + 1));
+          }
+          // ---- tile B: O_B += P_B(j) V(j), then S_B(j+1)
+          if (!(ok = wait_bar(bar(C::B_PFULL + 1), cnt & 1, ctl) && (shared || wait_full(vB(j))))) break;
+          tc_fence_after();
+          pv(1, vB(j), j == 0);
+          tc_commit(bar(C::B_EMPTY + vA(j) % C::NSTAGE));
+          if (!shared) tc_commit(bar(C::B_EMPTY + vB(j) % C::NSTAGE));
+          if (last) {
+            tc_commit(bar(C::B_OFINAL + 1));
+          } else {
+            qk(1, qB, kB(j + 1));
+            tc_commit(bar(C::B_EMPTY + kA(j + 1) % C::NSTAGE));
+            if (!shared) tc_commit(bar(C::B_EMPTY + kB(j + 1) % C::NSTAGE));
+            if (j + 1 == x.n_tiles - 1) tc_commit(bar(C::B_QEMPTY + qb));
+          }
+        }
+        ld += x.n_tiles * per;
+      }
+      if (*abort_flag) {
+        // Every MMA this thread issued must finish before TMEM is freed.
+        tc_commit(bar(C::B_DRAIN));
+        wait_bar(bar(C::B_DRAIN), 0, ctl, false);
+      }
+    }
+    __syncwarp();
+  }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    regs_inc<kSoftmaxRegs>();
+    const int half = warp >> 2;                      // 0: tile A, 1: tile B
+    const int r = tid & 127;                         // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_tmem = tmem + C::tmem_s(half) + lane_off;
+    const uint32_t o_tmem = tmem + C::tmem_o(half) + lane_off;
+    int cnt = 0, done_units = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      Unit x;
+      int hA;
+      unit_of(u, x, hA);
+      const int t = x.m0 + r;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < x.n_tiles; ++j, ++cnt) {
+        ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SFULL + half), cnt & 1, ctl));
+        if (!ok) break;
+        tc_fence_after();
+        float alpha;
+        const bool need = softmax_tile<F32>(s_tmem, x, j, t, a, m_run, l_run, alpha);
+        // O_X += P_X(j-1) V(j-1) has finished (it was issued before S_X(j)).
+        if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<D>(o_tmem, alpha);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + half));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_OFINAL + half), done_units & 1, ctl));
+      if (!ok) break;
+      ++done_units;
+      tc_fence_after();
+      store_row<D, OUT_F32>(o_tmem, a, x, hA + half, t, m_run, l_run);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+template <int D, bool F32, bool OUT_F32>
+cudaError_t launch_pair_impl(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, int grid, cudaStream_t stream) {
+  using C = PairCfg<D, F32>;
+  static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OUT_F32 || !F32, "fp32 inputs give fp32 outputs");
+  auto kern = swa_prefill_pair_kernel<D, F32, OUT_F32>;
+  // The register split inside the kernel assumes exactly kLaunchRegs per thread at launch;
+  // anything else could leave setmaxnreg.inc waiting, so refuse (the caller falls back).
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPairThreads, C::SMEM_BYTES, stream>>>(a, tq, tk, tv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_pair_supported(int Hq, int G, int d, bool f32) {
+  if (Hq % 2 != 0) return false;
+  const int tile = 128 * d * (f32 ? 4 : 2);
+  // The ring must hold two key tiles' slots: 2 slots per tile when the heads share
+  // a KV head, 4 otherwise (only the 8-slot ring of 16 KB tiles fits that).
+  return G % 2 == 0 || tile <= 16384;
+}
+
+cudaError_t launch_prefill_pair(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, int d, bool f32, bool out_f32, int grid,
+                                cudaStream_t stream) {
+  if (f32) {
+    if (d == 64) return launch_pair_impl<64, true, true>(a, tq, tk, tv, grid, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (out_f32) {
+    if (d == 64) return launch_pair_impl<64, false, true>(a, tq, tk, tv, grid, stream);
+    if (d == 128) return launch_pair_impl<128, false, true>(a, tq, tk, tv, grid, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (d == 64) return launch_pair_impl<64, false, false>(a, tq, tk, tv, grid, stream);
+  if (d == 128) return launch_pair_impl<128, false, false>(a, tq, tk, tv, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace swa

@@ -33,9 +33,21 @@ def rand_qkv(B, L, Hq, Hkv, d, seed, dtype=torch.bfloat16):
     return q, k, v
 
 
-def check_full(q, k, v, window, n_sink, what):
+class one_tile_kernel:
+    """Within the block, swa_fwd uses the one-query-tile kernel even where the
+    two-tile kernel applies (test hook, debug flag bit 1)."""
+
+    def __enter__(self):
+        self.prev = swa.swa_set_debug_flags(2)
+
+    def __exit__(self, *exc):
+        swa.swa_set_debug_flags(self.prev)
+
+
+def check_full(q, k, v, window, n_sink, what, both_kernels=True):
     """bf16 inputs are run twice: with fp32 output (the arithmetic, strict bound)
-    and with bf16 output (the bound plus the output's own rounding)."""
+    and with bf16 output (the bound plus the output's own rounding); and, where
+    the two-tile kernel applies, once more through the one-tile kernel."""
     scale = 1.0 / math.sqrt(q.shape[-1])
     ro, rl = oracle.swa_fwd(q, k, v, window, n_sink, scale)
     outs = [torch.float32] if q.dtype == torch.float32 else [torch.float32, torch.bfloat16]
@@ -43,6 +55,11 @@ def check_full(q, k, v, window, n_sink, what):
         out, lse = gpu_fwd(q, k, v, window, n_sink, scale, out_dtype=od)
         assert_close(out, ro, f"{what} out[{od}]")
         assert_close(lse, rl, f"{what} lse[{od}]")
+    if both_kernels:
+        with one_tile_kernel():
+            out, lse = gpu_fwd(q, k, v, window, n_sink, scale, out_dtype=outs[-1])
+        assert_close(out, ro, f"{what} out[one-tile kernel]")
+        assert_close(lse, rl, f"{what} lse[one-tile kernel]")
 
 
 def test_tiny_workload_fp32():
@@ -62,6 +79,11 @@ def test_tiny_workload_fp32():
     (3, 77, 4, 2, 128, 16, 4),         # a single partial tile per sequence
     (2, 1, 4, 4, 128, 8, 4),           # one token
     (1, 2048, 8, 8, 64, 128, 4),       # several q tiles, d = 64 with sinks
+    (2, 700, 3, 1, 128, 200, 4),       # odd head count (one-tile kernel only)
+    (1, 900, 6, 2, 128, 256, 4),       # G = 3: head pairs straddle KV heads
+    (1, 900, 6, 2, 64, 256, 4),        # same at d = 64 (two-tile kernel, separate K/V)
+    (4, 1024, 16, 16, 64, 128, 0),     # many units per CTA, d = 64, G = 1
+    (1, 4096, 32, 8, 128, 512, 4),     # many units per CTA, GQA
 ])
 def test_prefill_matches_oracle(B, L, Hq, Hkv, d, window, n_sink):
     q, k, v = rand_qkv(B, L, Hq, Hkv, d, seed=B * 1000 + L)
