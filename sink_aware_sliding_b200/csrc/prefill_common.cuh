@@ -125,6 +125,34 @@ __device__ __forceinline__ void build_varlen_tables(const PrefillArgs& a, int* s
 // writes P over S (packed bf16 pairs, or fp32 for the tf32 path) and updates
 // the running max and sum.  Returns whether the reference max moved; alpha is
 // the factor the row's O accumulator must be scaled by in that case.
+// Set the columns of s this row cannot see to -inf.  Visible: c <= hi and
+// (c >= lo or c < sk), all relative to the tile's first key.  The common edge
+// tiles need one compare per element: the diagonal tile (window start left of
+// the tile for every row of the warp) only the causal bound, the lower band
+// edge (tile end at or before every row's position) only the window bound; the
+// general predicate is left for tiles that touch the sink prefix.
+__device__ __forceinline__ void mask_tile(float* s, int hi, int lo, int sk) {
+  const bool no_lo = __all_sync(0xffffffffu, lo <= 0 || sk >= kBN);
+  const bool no_hi = __all_sync(0xffffffffu, hi >= kBN - 1);
+  const bool no_sink = __all_sync(0xffffffffu, sk <= 0);
+  if (no_lo) {
+#pragma unroll
+    for (int c = 0; c < kBN; ++c) s[c] = (c <= hi) ? s[c] : -INFINITY;
+  } else if (no_hi && no_sink) {
+#pragma unroll
+    for (int c = 0; c < kBN; ++c) s[c] = (c >= lo) ? s[c] : -INFINITY;
+  } else {
+#pragma unroll
+    for (int c = 0; c < kBN; ++c) s[c] = ((c <= hi) && (c >= lo || c < sk)) ? s[c] : -INFINITY;
+  }
+}
+
+// Online softmax of one key tile for the row this thread owns (TMEM lane).
+// Reads S from s_tmem (128 fp32 columns), masks it if the tile needs it,
+// moves the reference max only when it grew by more than 2^8 in exp2 units,
+// writes P over S (packed bf16 pairs, or fp32 for the tf32 path) and updates
+// the running max and sum.  Returns whether the reference max moved; alpha is
+// the factor the row's O accumulator must be scaled by in that case.
 template <bool F32>
 __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, const Unit& x, int j, int t,
                                              const PrefillArgs& a, float& m_run, float& l_run,
@@ -139,39 +167,38 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, const Unit& x, int
   }
   if (tile_needs_mask(x, j, a.window)) {
     const int n0 = tile_n0(x, j);
-    const int hi = t - n0;                 // visible: c <= hi
-    const int lo = t - a.window + 1 - n0;  //   and (c >= lo
-    const int sk = a.n_sink - n0;          //        or c < sk)
-#pragma unroll
-    for (int c = 0; c < kBN; ++c) {
-      const bool vis = (c <= hi) && (c >= lo || c < sk);
-      s[c] = vis ? s[c] : -INFINITY;
-    }
+    mask_tile(s, t - n0, t - a.window + 1 - n0, a.n_sink - n0);
   }
-  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+  // row max: 8 chains of three-input max
+  float mx[8];
 #pragma unroll
-  for (int c = 4; c < kBN; c += 4) {
-    mx0 = fmaxf(mx0, s[c]);
-    mx1 = fmaxf(mx1, s[c + 1]);
-    mx2 = fmaxf(mx2, s[c + 2]);
-    mx3 = fmaxf(mx3, s[c + 3]);
-  }
-  const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-  const float m_new = fmaxf(m_run, mx);
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[2 * i], s[2 * i + 1]);
+#pragma unroll
+  for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+  const float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+  const float m_new = fmaxf(m_run, m_tile);
   // NaN from (-inf) - (-inf) compares false: a row with nothing visible yet keeps -inf.
   const bool need = (m_new - m_run) * sl2 > 8.0f;
   const float m_use = need ? m_new : m_run;
   alpha = need ? ex2_approx((m_run - m_new) * sl2) : 1.0f;
   const float neg = (m_use == -INFINITY) ? 0.0f : -m_use * sl2;
-  float sum0 = 0.f, sum1 = 0.f;
+  // p = 2^(s * scale * log2 e - m * scale * log2 e): the argument on pairs, exp2 on the MUFU
+  const uint64_t scale2 = f2_pack(sl2, sl2), neg2 = f2_pack(neg, neg);
+  uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int c = 0; c < kBN; c += 2) {
-    s[c] = ex2_approx(fmaf(s[c], sl2, neg));
-    s[c + 1] = ex2_approx(fmaf(s[c + 1], sl2, neg));
-    sum0 += s[c];
-    sum1 += s[c + 1];
+  for (int i = 0; i < kBN / 2; ++i) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, neg2), x0, x1);
+    s[2 * i] = ex2_approx(x0);
+    s[2 * i + 1] = ex2_approx(x1);
+    acc[i & 3] = f2_add(acc[i & 3], f2_pack(s[2 * i], s[2 * i + 1]));
   }
-  l_run = l_run * alpha + (sum0 + sum1);
+  float sum0, sum1, sum2, sum3;
+  f2_unpack(f2_add(acc[0], acc[1]), sum0, sum1);
+  f2_unpack(f2_add(acc[2], acc[3]), sum2, sum3);
+  l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
   m_run = m_use;
   if constexpr (F32) {
 #pragma unroll
@@ -200,8 +227,14 @@ __device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {
   for (int c = 0; c < D / 32; ++c) {
     uint32_t rr[32];
     tmem_ld32_wait(o_tmem + c * 32, rr);
+    const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+    for (int i = 0; i < 16; ++i) {
+      float lo, hi;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1])), a2), lo, hi);
+      rr[2 * i] = __float_as_uint(lo);
+      rr[2 * i + 1] = __float_as_uint(hi);
+    }
     tmem_st32(o_tmem + c * 32, rr);
   }
 }
