@@ -279,6 +279,42 @@ __device__ __forceinline__ void store_row(uint32_t o_tmem, const PrefillArgs& a,
   }
 }
 
+// O / l of this thread's row, as bf16, into a 128-row x 128-byte shared tile in
+// the 128-byte swizzled layout the output tensor map stores from (d = 64), and
+// the row's LSE to global memory.
+__device__ __forceinline__ void stage_row_bf16_d64(uint32_t o_tmem, uint8_t* tile, int r,
+                                                   const PrefillArgs& a, const Unit& x, int h, int t,
+                                                   float m_run, float l_run) {
+  const float inv_l = 1.0f / l_run;
+  const uint64_t s2 = f2_pack(inv_l, inv_l);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t rr[32];
+    tmem_ld32_wait(o_tmem + c * 32, rr);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // 16-byte chunk 4c+q of the row: columns 32c+8q .. +7
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(rr[8 * q + 2 * e]), __uint_as_float(rr[8 * q + 2 * e + 1])), s2),
+                  lo, hi);
+        w[e] = pack_bf16x2(lo, hi);
+      }
+      const int chunk = 4 * c + q;
+      *reinterpret_cast<uint4*>(tile + r * 128 + ((chunk ^ (r & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (t < x.len && a.lse != nullptr) {
+    const size_t row = static_cast<size_t>(x.seq_start) + static_cast<size_t>(t);
+    const float ref = (m_run == -INFINITY) ? 0.0f : m_run * a.scale_log2;
+    const float lse = (ref + log2f(l_run)) * 0.69314718055994531f;
+    const size_t idx = a.lse_varlen ? static_cast<size_t>(h) * static_cast<size_t>(a.T) + row
+                                    : (static_cast<size_t>(x.seq) * a.Hq + h) * a.L + t;
+    a.lse[idx] = lse;
+  }
+}
+
 // Shared-memory matrix descriptors of the operands (see the kernels for the layouts).
 // K-major tile of `rows` rows x (NCHUNK x 128 bytes), 128-byte swizzle: MMA k-step kk of
 // 32 bytes lies in column chunk kk / steps_per_chunk.

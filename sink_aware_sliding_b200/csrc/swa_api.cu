@@ -103,8 +103,10 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
   int st = device_info(&dev);
   if (st != SWA_OK) return st;
   const bool f32 = dtype == SWA_DTYPE_F32;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
+  std::memset(&to, 0, sizeof(to));
   if ((st = make_map(&tq, q, f32, d, Hq, T, swa::kBM)) != SWA_OK) return st;
+  if (dtype == SWA_DTYPE_BF16 && (st = make_map(&to, out, false, d, Hq, T, swa::kBM)) != SWA_OK) return st;
   if ((st = make_map(&tk, k, f32, d, Hkv, T, swa::kBN)) != SWA_OK) return st;
   if ((st = make_map(&tv, v, f32, d, Hkv, T, swa::kBN, f32)) != SWA_OK) return st;
   swa::PrefillArgs a{};
@@ -142,7 +144,7 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
   const int grid = static_cast<int>(std::min<long long>(dev->sms, units));
   if (grid <= 0) return SWA_OK;
   cudaError_t e = cudaErrorNotSupported;
-  if (pair) e = swa::launch_prefill_pair(a, tq, tk, tv, d, f32, dtype != SWA_DTYPE_BF16, grid, stream);
+  if (pair) e = swa::launch_prefill_pair(a, tq, tk, tv, to, d, f32, dtype != SWA_DTYPE_BF16, grid, stream);
   if (e == cudaErrorNotSupported) {  // one-tile kernel (odd Hq, or the two-tile kernel declined)
     const int grid1 = static_cast<int>(std::min<long long>(dev->sms, pair ? 2 * units : units));
     e = swa::launch_prefill(a, tq, tk, tv, d, f32, dtype != SWA_DTYPE_BF16, grid1, stream);

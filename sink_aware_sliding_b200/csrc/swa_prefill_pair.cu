@@ -20,6 +20,10 @@
 // ready implies O_X += P_X(j) V(j) has finished, so a softmax warp may rescale
 // its O rows right after reading S without a further barrier.
 // TMEM columns: S_A 0-127, S_B 128-255, O_A 256.., O_B 256+D.. (512 allocated).
+// With d = 64 and bf16 output, a unit's finished Q tiles double as the staging
+// tiles of its output: each softmax warpgroup writes its normalised O rows there
+// in the swizzled layout and one thread stores the tile with TMA; the Q buffer is
+// handed back to the load warp only after both stores have read it.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -69,6 +73,7 @@ struct PairCfg {
   static constexpr int SMEM_BYTES = OFF_TABLES + 2 * 4 * (kMaxSeqSmem + 1) + 1024;
   static constexpr uint32_t IDESC_QK = make_idesc(F32 ? 2u : 1u, kBM, kBN, false);
   static constexpr uint32_t IDESC_PV = make_idesc(F32 ? 2u : 1u, kBM, D, true);
+  static constexpr bool TMA_STORE = !F32 && D == 64;   // requires QBUF == 2 (see above)
   __device__ static constexpr uint32_t tmem_s(int half) { return half ? 128u : 0u; }
   __device__ static constexpr uint32_t tmem_o(int half) { return 256u + (half ? D : 0); }
 };
@@ -76,8 +81,11 @@ struct PairCfg {
 template <int D, bool F32, bool OUT_F32>
 __global__ void __launch_bounds__(kPairThreads, 1)
     swa_prefill_pair_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
-                            const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+                            const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                            const __grid_constant__ CUtensorMap to) {
   using C = PairCfg<D, F32>;
+  constexpr bool kTmaStore = C::TMA_STORE && !OUT_F32;
+  static_assert(!kTmaStore || C::QBUF == 2, "output staging reuses the previous unit's Q buffer");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -96,7 +104,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < C::QBUF; ++i) {
       mbar_init(bar(C::B_QFULL + i), 1);
-      mbar_init(bar(C::B_QEMPTY + i), 1);
+      // freed by the MMA warp (tcgen05.commit), or by both epilogues after their stores
+      mbar_init(bar(C::B_QEMPTY + i), kTmaStore ? 2 : 1);
     }
     for (int i = 0; i < C::NSTAGE; ++i) {
       mbar_init(bar(C::B_FULL + i), 1);
@@ -115,6 +124,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    if (kTmaStore) tma_prefetch_desc(&to);
   }
   if (a.cu_seqlens != nullptr && warp == 0) build_varlen_tables(a, s_cu, s_tpre, lane);
   if (warp == kMmaWarp) {
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         qk(1, qB, kB(0));
         tc_commit(bar(C::B_EMPTY + kA(0) % C::NSTAGE));
         if (!shared) tc_commit(bar(C::B_EMPTY + kB(0) % C::NSTAGE));
-        if (x.n_tiles == 1) tc_commit(bar(C::B_QEMPTY + qb));
+        if (!kTmaStore && x.n_tiles == 1) tc_commit(bar(C::B_QEMPTY + qb));
         for (int j = 0; j < x.n_tiles; ++j, ++cnt) {
           const bool last = j == x.n_tiles - 1;
           // ---- tile A: O_A += P_A(j) V(j), then S_A(j+1)
@@ -260,7 +270,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             qk(1, qB, kB(j + 1));
             tc_commit(bar(C::B_EMPTY + kA(j + 1) % C::NSTAGE));
             if (!shared) tc_commit(bar(C::B_EMPTY + kB(j + 1) % C::NSTAGE));
-            if (j + 1 == x.n_tiles - 1) tc_commit(bar(C::B_QEMPTY + qb));
+            if (!kTmaStore && j + 1 == x.n_tiles - 1) tc_commit(bar(C::B_QEMPTY + qb));
           }
         }
         ld += x.n_tiles * per;
@@ -284,6 +294,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     int cnt = 0, done_units = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const int qb = done_units % C::QBUF;
       Unit x;
       int hA;
       unit_of(u, x, hA);
@@ -306,8 +317,29 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (!ok) break;
       ++done_units;
       tc_fence_after();
-      store_row<D, OUT_F32>(o_tmem, a, x, hA + half, t, m_run, l_run);
+      if constexpr (kTmaStore) {
+        // Every MMA that read this unit's Q tiles finished before O_X was final.
+        const uint32_t tile = base + C::OFF_Q + (qb * 2 + half) * C::TILE;
+        if (x.m1 - x.m0 == kBM - 1) {
+          stage_row_bf16_d64(o_tmem, gbase + (tile - base), r, a, x, hA + half, t, m_run, l_run);
+          fence_proxy_async_smem();
+          named_bar_sync(1 + half, 128);
+          if (r == 0) {
+            tma_store_3d(&to, tile, 0, hA + half, x.seq_start + x.m0);
+            bulk_commit();
+            bulk_wait_read();
+            mbar_arrive(bar(C::B_QEMPTY + qb));
+          }
+        } else {
+          store_row<D, OUT_F32>(o_tmem, a, x, hA + half, t, m_run, l_run);
+          named_bar_sync(1 + half, 128);
+          if (r == 0) mbar_arrive(bar(C::B_QEMPTY + qb));
+        }
+      } else {
+        store_row<D, OUT_F32>(o_tmem, a, x, hA + half, t, m_run, l_run);
+      }
     }
+    if (kTmaStore && r == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -318,7 +350,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
 template <int D, bool F32, bool OUT_F32>
 cudaError_t launch_pair_impl(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, int grid, cudaStream_t stream) {
+                             const CUtensorMap& tv, const CUtensorMap& to, int grid, cudaStream_t stream) {
   using C = PairCfg<D, F32>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(OUT_F32 || !F32, "fp32 inputs give fp32 outputs");
@@ -331,7 +363,7 @@ cudaError_t launch_pair_impl(const PrefillArgs& a, const CUtensorMap& tq, const 
   if (fa.numRegs != kLaunchRegs) return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPairThreads, C::SMEM_BYTES, stream>>>(a, tq, tk, tv);
+  kern<<<grid, kPairThreads, C::SMEM_BYTES, stream>>>(a, tq, tk, tv, to);
   return cudaGetLastError();
 }
 
@@ -346,19 +378,19 @@ bool prefill_pair_supported(int Hq, int G, int d, bool f32) {
 }
 
 cudaError_t launch_prefill_pair(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, int d, bool f32, bool out_f32, int grid,
-                                cudaStream_t stream) {
+                                const CUtensorMap& tv, const CUtensorMap& to, int d, bool f32,
+                                bool out_f32, int grid, cudaStream_t stream) {
   if (f32) {
-    if (d == 64) return launch_pair_impl<64, true, true>(a, tq, tk, tv, grid, stream);
+    if (d == 64) return launch_pair_impl<64, true, true>(a, tq, tk, tv, to, grid, stream);
     return cudaErrorInvalidValue;
   }
   if (out_f32) {
-    if (d == 64) return launch_pair_impl<64, false, true>(a, tq, tk, tv, grid, stream);
-    if (d == 128) return launch_pair_impl<128, false, true>(a, tq, tk, tv, grid, stream);
+    if (d == 64) return launch_pair_impl<64, false, true>(a, tq, tk, tv, to, grid, stream);
+    if (d == 128) return launch_pair_impl<128, false, true>(a, tq, tk, tv, to, grid, stream);
     return cudaErrorInvalidValue;
   }
-  if (d == 64) return launch_pair_impl<64, false, false>(a, tq, tk, tv, grid, stream);
-  if (d == 128) return launch_pair_impl<128, false, false>(a, tq, tk, tv, grid, stream);
+  if (d == 64) return launch_pair_impl<64, false, false>(a, tq, tk, tv, to, grid, stream);
+  if (d == 128) return launch_pair_impl<128, false, false>(a, tq, tk, tv, to, grid, stream);
   return cudaErrorInvalidValue;
 }
 
