@@ -228,3 +228,34 @@ def ring_append(kc, vc, sk, sv, k_new, v_new, pos, window: int, n_sink: int) -> 
         if p < n_sink:
             sk[b, :, p] = k_new[b]
             sv[b, :, p] = v_new[b]
+
+
+# ---------------------------------------------------------------------------
+# Hadamard output projection ("Rethinking Attention Output Projection:
+# Structured Hadamard Transforms for Efficient Transformers", section 2,
+# Methodology): MHA_Had(X) = alpha * (Y H) + beta, with H the fixed Walsh-
+# Hadamard matrix, which preserves the l2 norm (so it is orthonormal).
+# Reading: H is the Sylvester-ordered matrix of size n = Hq * d (a power of two),
+# H[i, j] = (-1)^popcount(i & j) / sqrt(n); Y is one token's attention output
+# with the heads concatenated (head-major, h * d + c).
+# ---------------------------------------------------------------------------
+
+def hadamard_matrix(n: int) -> np.ndarray:
+    """Sylvester Walsh-Hadamard matrix of size n, normalised to be orthonormal."""
+    if n < 1 or n & (n - 1):
+        raise ValueError("n must be a power of two")
+    i = np.arange(n, dtype=np.int64)
+    bits = np.bitwise_and(i[:, None], i[None, :])
+    pop = np.zeros_like(bits)
+    while bits.any():
+        pop += bits & 1
+        bits >>= 1
+    return np.where(pop % 2 == 0, 1.0, -1.0) / np.sqrt(n)
+
+
+def hadamard_proj(y, alpha, beta) -> np.ndarray:
+    """alpha * (y @ H) + beta for rows y [N, n] (any float input), in float64."""
+    y = _f64(y)
+    n = y.shape[-1]
+    H = hadamard_matrix(n)
+    return _f64(alpha) * (y.reshape(-1, n) @ H).reshape(y.shape) + _f64(beta)
