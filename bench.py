@@ -10,7 +10,8 @@ L=2048, d=64, window 128), counting 4*d FLOPs per visible (query, key) pair.
 The same line carries, under "workloads", the other workloads measured the
 same way: the 8B-shaped GQA prefill and the packed long-context prefill
 (TFLOP/s against the tensor roofline) and the ring-buffer decode (HBM GB/s and
-tokens/s against the HBM roofline).
+tokens/s against the HBM roofline) and the Hadamard output projection of the
+GQA prefill's output (HBM GB/s).
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -341,6 +342,71 @@ def bench_prefill(name, steps, warmup, dev, flush, peaks, sampler):
     }
 
 
+def bench_hadamard(name, steps, warmup, dev, flush, peaks, sampler):
+    """Hadamard output projection over T token rows: read y (bf16), write z (bf16)."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    w = wl.PROJ_WORKLOADS[name]
+    y, alpha, beta = wl.make_hadamard(w, device=dev)
+    z = torch.empty_like(y)
+
+    def run(yy=y, zz=z):
+        swa.swa_hadamard_proj(yy, alpha, beta, zz)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    alg_bytes = 2 * w.T * w.n * 2 + 2 * w.n * 4
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+
+    hy = y.cpu().pin_memory()
+    hz = torch.empty(z.shape, dtype=z.dtype).pin_memory()
+    dy = torch.empty_like(y)
+
+    def e2e_step():
+        dy.copy_(hy, non_blocking=True)
+        run(dy, z)
+        hz.copy_(z, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(3, steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "traffic": profiled_traffic(name), "algorithmic_bytes_per_launch": alg_bytes}
+    return {
+        "config": w.describe(), "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
+        "tokens_per_s": round(w.T / (ms * 1e-3), 1), "roofline": roof,
+        "e2e": {"value": round(alg_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": y.numel() * 2,
+                "d2h_bytes_per_step": z.numel() * 2},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
 def bench_decode(name, steps, warmup, dev, peaks, sampler):
     """One step = one generated token for all B sequences: cache append + split-K decode + merge."""
     import torch
@@ -500,8 +566,16 @@ def profile_case(args):
     import workloads as wl
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = wl.WORKLOADS[args.profile_case]
     n = args.warmup + args.steps
+    if args.profile_case in wl.PROJ_WORKLOADS:
+        pw = wl.PROJ_WORKLOADS[args.profile_case]
+        y, alpha, beta = wl.make_hadamard(pw, device=dev, T=args.L)
+        z = torch.empty_like(y)
+        for _ in range(n):
+            swa.swa_hadamard_proj(y, alpha, beta, z)
+        torch.cuda.synchronize()
+        return
+    w = wl.WORKLOADS[args.profile_case]
     if w.kind == "prefill":
         q, k, v = wl.make_prefill(w, device=dev, B=args.B, L=args.L)
         out = torch.empty_like(q)
@@ -542,7 +616,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
-    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode")
+    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,hadamard_proj")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -590,6 +664,8 @@ def main():
     for n in names:
         if n == "decode":
             results[n] = bench_decode(n, args.decode_tokens, args.warmup, dev, peaks, sampler)
+        elif n == "hadamard_proj":
+            results[n] = bench_hadamard(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         else:
             results[n] = bench_prefill(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         torch.cuda.empty_cache()

@@ -165,6 +165,23 @@ int swa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                        int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
                        swa_stream_t stream);
 
+/*
+ * Hadamard output projection, the step after attention ("Rethinking Attention
+ * Output Projection: Structured Hadamard Transforms for Efficient Transformers",
+ * section 2): per row, z = alpha * (y H) + beta, where H is the fixed Walsh-
+ * Hadamard matrix, which preserves the l2 norm.  Reading used: H is the
+ * Sylvester-ordered matrix of size n normalised by 1/sqrt(n),
+ * H[i][j] = (-1)^popcount(i & j) / sqrt(n), computed as a fast Walsh-Hadamard
+ * transform; y is a row of attention output with the heads concatenated
+ * (n = Hq * d, the [.., Hq, d] layout of swa_fwd / swa_decode outputs).
+ *   y     [n_rows, n] bf16              (read)
+ *   alpha, beta [n]   float32           (read; the learned rescaling)
+ *   z     [n_rows, n] bf16 or float32 per out_dtype (SWA_DTYPE_BF16 / SWA_DTYPE_F32)
+ * Supported: n a power of two with 32 <= n <= 8192.  fp32 arithmetic.
+ */
+int swa_hadamard_proj(const void* y, const float* alpha, const float* beta, void* z,
+                      long long n_rows, int n, int out_dtype, swa_stream_t stream);
+
 /* Static text for a status code. */
 const char* swa_status_string(int status);
 

@@ -36,6 +36,7 @@ EXPORTS = (
     "swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append",
     "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
+    "swa_hadamard_proj",
 )
 
 _lib = None
@@ -63,6 +64,7 @@ def _load():
     lib.swa_decode_workspace_bytes.restype = SZ
     lib.swa_decode.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.swa_hadamard_proj.argtypes = [P, P, P, P, LL, I, I, P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
@@ -70,7 +72,7 @@ def _load():
     lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
-                 "swa_decode_noalloc",
+                 "swa_decode_noalloc", "swa_hadamard_proj",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -203,6 +205,23 @@ def swa_decode_noalloc(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window:
                                     _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window),
                                     int(n_sink), _scale(scale, d), _stream(stream))
     _check(st, "swa_decode_noalloc")
+
+
+def swa_hadamard_proj(y, alpha, beta, z, stream=None) -> None:
+    """z = alpha * (y H) + beta per row of n = alpha.numel() elements; y bf16 holding a
+    whole number of rows in any contiguous shape (e.g. an attention output [T, Hq, d]
+    with n = Hq * d), z of the same shape in bf16 or float32, alpha/beta [n] float32.
+    H is the orthonormal Walsh-Hadamard matrix of size n."""
+    import torch
+    n = alpha.numel()
+    _need(y.dtype == torch.bfloat16 and y.is_contiguous() and z.is_contiguous(), "y bf16 contiguous")
+    _need(z.shape == y.shape, "z shape")
+    _need(alpha.dtype == beta.dtype == torch.float32 and beta.numel() == n, "alpha/beta float32 [n]")
+    _need(n > 0 and y.numel() % n == 0, "y holds a whole number of rows of n")
+    code = SWA_DTYPE_F32 if z.dtype == torch.float32 else SWA_DTYPE_BF16
+    st = _load().swa_hadamard_proj(_ptr(y), _ptr(alpha), _ptr(beta), _ptr(z), y.numel() // n, n, code,
+                                   _stream(stream))
+    _check(st, "swa_hadamard_proj")
 
 
 def swa_device_error(stream=None) -> int:

@@ -303,6 +303,20 @@ int swa_decode(const void* q, const void* kcache, const void* vcache, const void
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+int swa_hadamard_proj(const void* y, const float* alpha, const float* beta, void* z,
+                      long long n_rows, int n, int out_dtype, swa_stream_t stream) {
+  if (n_rows < 0 || n < 32 || n > 8192 || (n & (n - 1)) != 0) return n_rows < 0 ? SWA_ERR_INVALID_ARG
+                                                                      : SWA_ERR_UNSUPPORTED;
+  if (out_dtype != SWA_DTYPE_BF16 && out_dtype != SWA_DTYPE_F32) return SWA_ERR_INVALID_ARG;
+  if (n_rows == 0) return SWA_OK;
+  if (!y || !alpha || !beta || !z || !aligned16(y) || !aligned16(alpha) || !aligned16(beta) ||
+      !aligned16(z))
+    return SWA_ERR_INVALID_ARG;
+  cudaError_t e = swa::launch_hadamard(y, alpha, beta, z, n_rows, n, out_dtype == SWA_DTYPE_F32,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 const char* swa_status_string(int status) {
   switch (status) {
     case SWA_OK: return "ok";

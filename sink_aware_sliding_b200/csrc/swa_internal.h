@@ -68,4 +68,8 @@ cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* pos
                                 void* vc, void* sk, void* sv, int B, int Hkv, int d, int W, int S,
                                 cudaStream_t stream);
 
+// Hadamard output projection z = alpha * (y H) + beta over rows of n = 2^k elements.
+cudaError_t launch_hadamard(const void* y, const float* alpha, const float* beta, void* z,
+                            long long n_rows, int n, bool out_f32, cudaStream_t stream);
+
 }  // namespace swa

@@ -28,16 +28,23 @@ def assert_close(got, want, what: str, max_abs: float = MAX_ABS, mean_abs: float
     When ``got`` is a bf16 tensor, each element may in addition differ by the
     half-ulp of rounding the exact value to bf16: a bf16 output cannot hold the
     oracle's value more closely than that (half an ulp is 0.0156 at |x| in [4, 8),
-    above the 1e-2 bound by itself).
+    above the 1e-2 bound by itself).  The mean bound takes the mean of the same
+    allowance: if the fp32 result g32 meets mean|g32 - want| <= mean_abs, then
+    bf16(g32) meets mean|bf16(g32) - want| <= mean_abs + mean(half-ulp), and
+    nothing tighter holds for O(1) outputs, whose rounding alone averages about
+    a quarter ulp (0.002 at |x| near 1.5).  The strict bounds are checked on the
+    fp32-output modes of the same kernels.
     """
     out_bf16 = hasattr(got, "dtype") and got.dtype == torch.bfloat16
     g, w = to64(got), to64(want)
     assert g.shape == w.shape, f"{what}: shape {g.shape} vs {w.shape}"
     assert np.isfinite(g).all(), f"{what}: non-finite values"
     err = np.abs(g - w)
-    allow = max_abs + (bf16_half_ulp(w) if out_bf16 else 0.0)
+    hu = bf16_half_ulp(w) if out_bf16 else np.zeros_like(w)
+    allow = max_abs + hu
     excess = float((err - allow).max()) if err.size else -1.0
     mx, mn = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
-    assert excess <= 0 and mn <= mean_abs, (
+    mean_allow = mean_abs + (float(hu.mean()) if err.size else 0.0)
+    assert excess <= 0 and mn <= mean_allow, (
         f"{what}: max_abs={mx:.3e} (allowance exceeded by {excess:.3e}) mean_abs={mn:.3e}")
     return mx, mn

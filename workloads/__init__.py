@@ -232,3 +232,35 @@ def sample_rows(L: int, window: int, n_sink: int, block: int = 128, n_random: in
     if L > 0:
         rows.update(torch.randint(0, L, (n_random,), generator=g).tolist())
     return sorted(rows)
+
+
+@dataclasses.dataclass(frozen=True)
+class ProjWorkload:
+    """Output projection after attention: T token rows of n = Hq * d features."""
+    name: str
+    T: int
+    n: int
+    out_dtype: str = "bf16"
+    note: str = ""
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "kind": "hadamard_proj", "T": self.T, "n": self.n,
+                "in_dtype": "bf16", "out_dtype": self.out_dtype}
+
+
+PROJ_WORKLOADS = {
+    "hadamard_proj": ProjWorkload(
+        "hadamard_proj", T=32768, n=4096,
+        note="Hadamard output projection of the 8B-shaped prefill's attention output (32 x 128)"),
+}
+
+
+def make_hadamard(w: ProjWorkload, device="cpu", T: Optional[int] = None):
+    """y [T, n] bf16 from N(0, 1); alpha [n] = 1 + 0.5 N(0, 1); beta [n] = 0.1 N(0, 1) (fp32),
+    drawn in that order from the seed-0 generator."""
+    T = w.T if T is None else T
+    g = _gen(device)
+    y = _normal(g, (T, w.n), device).to(torch.bfloat16)
+    alpha = 1.0 + 0.5 * _normal(g, (w.n,), device)
+    beta = 0.1 * _normal(g, (w.n,), device)
+    return y, alpha, beta
