@@ -312,7 +312,19 @@ int swa_hadamard_proj(const void* y, const float* alpha, const float* beta, void
   if (!y || !alpha || !beta || !z || !aligned16(y) || !aligned16(alpha) || !aligned16(beta) ||
       !aligned16(z))
     return SWA_ERR_INVALID_ARG;
-  cudaError_t e = swa::launch_hadamard(y, alpha, beta, z, n_rows, n, out_dtype == SWA_DTYPE_F32,
+  DeviceInfo* di = nullptr;
+  const int st = device_info(&di);
+  if (st != SWA_OK) return st;
+  swa::HadamardArgs a;
+  a.y = y;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.z = z;
+  a.n_rows = n_rows;
+  a.timeout_ns = g_timeout_ns.load();
+  a.debug_flags = g_debug_flags.load();
+  a.err = di->err;
+  cudaError_t e = swa::launch_hadamard(a, n, out_dtype == SWA_DTYPE_F32, di->sms,
                                        reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }

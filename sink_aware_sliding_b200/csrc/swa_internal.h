@@ -69,7 +69,16 @@ cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* pos
                                 cudaStream_t stream);
 
 // Hadamard output projection z = alpha * (y H) + beta over rows of n = 2^k elements.
-cudaError_t launch_hadamard(const void* y, const float* alpha, const float* beta, void* z,
-                            long long n_rows, int n, bool out_f32, cudaStream_t stream);
+struct HadamardArgs {
+  const void* y;            // [n_rows, n] bf16
+  const float* alpha;       // [n]
+  const float* beta;        // [n]
+  void* z;                  // [n_rows, n] bf16 or f32
+  long long n_rows;
+  unsigned long long timeout_ns;
+  int debug_flags;          // bit 0: issue no loads (the waits then time out)
+  int* err;                 // device status word (first error wins)
+};
+cudaError_t launch_hadamard(const HadamardArgs& a, int n, bool out_f32, int sms, cudaStream_t stream);
 
 }  // namespace swa

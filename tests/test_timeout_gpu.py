@@ -44,3 +44,4 @@ def test_expired_wait_reports_timeout_and_context_survives(one_tile):
     ro, rl = oracle.swa_fwd(q, k, v, 128, 4, 1 / math.sqrt(128))
     assert_close(out, ro, "after timeout: out")
     assert_close(lse, rl, "after timeout: lse")
+
