@@ -7,7 +7,8 @@ library never calls it, imports nothing from it and shares no code with it.
 The arithmetic lives in ``swa_oracle.c`` (plain C, double precision, OpenMP
 over query rows); this module only marshals numpy arrays through ctypes and
 holds the plain model of the ring-buffer KV cache (slot bookkeeping, no
-arithmetic on values).
+arithmetic on values), the Hadamard output projection and the rotary position
+encoding, both in numpy float64.
 
 Parity pins: every function here is checked by the ``-m "not gpu"`` tests
 against closed forms, a library causal-attention routine, brute-force masks
@@ -259,3 +260,39 @@ def hadamard_proj(y, alpha, beta) -> np.ndarray:
     n = y.shape[-1]
     H = hadamard_matrix(n)
     return _f64(alpha) * (y.reshape(-1, n) @ H).reshape(y.shape) + _f64(beta)
+
+
+# ---------------------------------------------------------------------------
+# Rotary position encoding on the sliding-window branch ("Simple linear
+# attention language models balance the recall-throughput tradeoff", proposed
+# method: the window attention uses rotary position encoding, the linear branch
+# none).  The page gives no formula; reading used: the RoFormer rotation with
+# the rotate-half pairing.  For i < d/2 the pair (x[i], x[i + d/2]) of a vector
+# at absolute position p turns by the angle p * theta_i, theta_i =
+# base^(-2i/d):
+#     x'[i]       = x[i] cos(p theta_i) - x[i + d/2] sin(p theta_i)
+#     x'[i + d/2] = x[i] sin(p theta_i) + x[i + d/2] cos(p theta_i)
+# Positions are absolute token positions (a cached key keeps the rotation of
+# its own position; nothing is re-indexed inside the window).
+# ---------------------------------------------------------------------------
+
+def rope_angles(positions, d: int, base: float) -> np.ndarray:
+    """Angles p * base^(-2i/d), shape [len(positions), d/2], float64."""
+    if d < 2 or d % 2:
+        raise ValueError("d must be even")
+    p = np.asarray(positions, dtype=np.float64).reshape(-1)
+    theta = np.power(float(base), -2.0 * np.arange(d // 2, dtype=np.float64) / d)
+    return p[:, None] * theta[None, :]
+
+
+def rope(x, positions, base: float = 10000.0) -> np.ndarray:
+    """Rotate x [N, ..., d] (any float input) at positions [N]; float64 result."""
+    x = _f64(x)
+    d = x.shape[-1]
+    ang = rope_angles(positions, d, base)                     # [N, d/2]
+    if ang.shape[0] != x.shape[0]:
+        raise ValueError("one position per leading index")
+    shape = (x.shape[0],) + (1,) * (x.ndim - 2) + (d // 2,)
+    c, s = np.cos(ang).reshape(shape), np.sin(ang).reshape(shape)
+    lo, hi = x[..., : d // 2], x[..., d // 2:]
+    return np.concatenate([lo * c - hi * s, lo * s + hi * c], axis=-1)
