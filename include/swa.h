@@ -166,6 +166,48 @@ int swa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                        swa_stream_t stream);
 
 /*
+ * Rotary position encoding of the sliding-window branch ("Simple linear
+ * attention language models balance the recall-throughput tradeoff", proposed
+ * method: the window attention uses rotary position encoding, the linear branch
+ * none).  The page gives no formula; reading used: the RoFormer rotation with
+ * rotate-half pairs.  For i < d/2 the pair (x[i], x[i + d/2]) of a vector at
+ * absolute position p turns by the angle p * theta_i, theta_i =
+ * rope_base^(-2i/d) (10000 is the usual base):
+ *   x'[i] = x[i] cos - x[i+d/2] sin,   x'[i+d/2] = x[i] sin + x[i+d/2] cos.
+ * The angle is formed in double precision and reduced to [-pi, pi] before a
+ * single-precision sine/cosine; the rotated values are rounded to bf16 (RNE).
+ * A cached key keeps the rotation of its own position; nothing is re-indexed
+ * inside the window.  Supported d: 64, 128.  rope_base > 0 and finite.
+ *
+ * swa_rope_qk: rotates in place q [n_tokens, Hq, d] and k [n_tokens, Hkv, d]
+ * (bf16, device, 16-byte aligned; k may be NULL to rotate q alone, or Hq = 0
+ * to rotate k alone), token t at positions[t] (int32, device).  Used before
+ * swa_fwd / swa_fwd_varlen, whose kernels take rotated q and k.
+ */
+int swa_rope_qk(void* q, void* k, const int32_t* positions, long long n_tokens, int Hq, int Hkv, int d,
+                double rope_base, swa_stream_t stream);
+
+/*
+ * swa_cache_append with the new key rotated at pos[b] first (one launch): the
+ * decode step's "rotate k on append".  Arguments as swa_cache_append plus
+ * rope_base; v_new is stored unchanged.
+ */
+int swa_rope_cache_append(const void* k_new, const void* v_new, const int32_t* pos, void* kcache,
+                          void* vcache, void* sink_k, void* sink_v, int B, int Hkv, int d, int window,
+                          int n_sink, double rope_base, swa_stream_t stream);
+
+/*
+ * swa_decode with the query rotated at pos[b] inside the decode kernel (the
+ * decode step's "rotate q"); the cache must hold rotated keys (swa_rope_qk
+ * before swa_cache_fill, swa_rope_cache_append per step).  Arguments, workspace
+ * (same size as swa_decode's) and errors as swa_decode, plus rope_base.
+ */
+int swa_decode_rope(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                    const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
+                    int Hkv, int d, int window, int n_sink, float scale, double rope_base,
+                    void* workspace, size_t workspace_bytes, swa_stream_t stream);
+
+/*
  * Hadamard output projection, the step after attention ("Rethinking Attention
  * Output Projection: Structured Hadamard Transforms for Efficient Transformers",
  * section 2): per row, z = alpha * (y H) + beta, where H is the fixed Walsh-

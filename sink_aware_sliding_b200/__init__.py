@@ -36,7 +36,7 @@ EXPORTS = (
     "swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append",
     "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
-    "swa_hadamard_proj",
+    "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope",
 )
 
 _lib = None
@@ -65,6 +65,10 @@ def _load():
     lib.swa_decode.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.swa_hadamard_proj.argtypes = [P, P, P, P, LL, I, I, P]
+    D = ctypes.c_double
+    lib.swa_rope_qk.argtypes = [P, P, P, LL, I, I, I, D, P]
+    lib.swa_rope_cache_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P]
+    lib.swa_decode_rope.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, D, P, SZ, P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
@@ -72,7 +76,8 @@ def _load():
     lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
-                 "swa_decode_noalloc", "swa_hadamard_proj",
+                 "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
+                 "swa_decode_rope",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -177,6 +182,34 @@ def swa_cache_append(k_new, v_new, pos, kcache, vcache, sink_k, sink_v, window: 
     _check(st, "swa_cache_append")
 
 
+def swa_rope_cache_append(k_new, v_new, pos, kcache, vcache, sink_k, sink_v, window: int, n_sink: int,
+                          rope_base: float = 10000.0, stream=None) -> None:
+    """swa_cache_append with k_new rotated at pos[b] (rotary encoding) before it is stored."""
+    B, Hkv, d = k_new.shape
+    st = _load().swa_rope_cache_append(_ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(kcache), _ptr(vcache),
+                                       _ptr(sink_k), _ptr(sink_v), B, Hkv, d, int(window), int(n_sink),
+                                       float(rope_base), _stream(stream))
+    _check(st, "swa_rope_cache_append")
+
+
+def swa_rope_qk(q, k, positions, rope_base: float = 10000.0, stream=None) -> None:
+    """Rotate q [..., Hq, d] and k [..., Hkv, d] (bf16, contiguous; k may be None) in place;
+    the leading dimensions flatten to tokens, token t at positions[t] (int32, device)."""
+    import torch
+    _need(q.dtype == torch.bfloat16 and q.is_contiguous(), "q bf16 contiguous")
+    Hq, d = q.shape[-2], q.shape[-1]
+    T = q.numel() // (Hq * d)
+    Hkv = 0
+    if k is not None:
+        _need(k.dtype == torch.bfloat16 and k.is_contiguous() and k.shape[-1] == d, "k bf16 contiguous")
+        Hkv = k.shape[-2]
+        _need(k.numel() == T * Hkv * d, "k tokens")
+    _need(positions.dtype == torch.int32 and positions.numel() == T, "positions int32 [T]")
+    st = _load().swa_rope_qk(_ptr(q), _ptr(k) if k is not None else None, _ptr(positions), T, Hq, Hkv, d,
+                             float(rope_base), _stream(stream))
+    _check(st, "swa_rope_qk")
+
+
 def swa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, window: int, n_sink: int) -> int:
     return int(_load().swa_decode_workspace_bytes(B, Hq, Hkv, d, window, n_sink))
 
@@ -191,6 +224,18 @@ def swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_
                             _scale(scale, d), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream))
     _check(st, "swa_decode")
+
+
+def swa_decode_rope(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,
+                    workspace, rope_base: float = 10000.0, scale=None, stream=None) -> None:
+    """swa_decode with q rotated at pos[b] inside the kernel (the cache holds rotated keys)."""
+    B, Hq, d = q.shape
+    Hkv = kcache.shape[1]
+    st = _load().swa_decode_rope(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(sink_k), _ptr(sink_v),
+                                 _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window), int(n_sink),
+                                 _scale(scale, d), float(rope_base), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "swa_decode_rope")
 
 
 def swa_decode_noalloc(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,

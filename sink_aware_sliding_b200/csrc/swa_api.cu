@@ -259,10 +259,10 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int window, int
   return slots * swa::decode_partial_floats(Hq / Hkv, d) * sizeof(float);
 }
 
-int swa_decode(const void* q, const void* kcache, const void* vcache, const void* sink_k,
-               const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
-               int Hkv, int d, int window, int n_sink, float scale, void* workspace,
-               size_t workspace_bytes, swa_stream_t stream) {
+static int run_decode(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                      const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
+                      int Hkv, int d, int window, int n_sink, float scale, void* workspace,
+                      size_t workspace_bytes, const swa::RopeTable* rope, swa_stream_t stream) {
   int st = decode_shape_ok(B, Hq, Hkv, d, window, n_sink);
   if (st != SWA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
@@ -299,7 +299,61 @@ int swa_decode(const void* q, const void* kcache, const void* vcache, const void
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_warps = grid * (swa::decode_threads() / 32);
   cudaError_t e = swa::launch_decode(a, d, grid, swa::decode_threads(),
-                                     reinterpret_cast<cudaStream_t>(stream));
+                                     reinterpret_cast<cudaStream_t>(stream), rope);
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_decode(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+               const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
+               int Hkv, int d, int window, int n_sink, float scale, void* workspace,
+               size_t workspace_bytes, swa_stream_t stream) {
+  return run_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
+                    scale, workspace, workspace_bytes, nullptr, stream);
+}
+
+static bool rope_base_ok(double base) { return base > 0.0 && std::isfinite(base); }
+
+int swa_decode_rope(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                    const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
+                    int Hkv, int d, int window, int n_sink, float scale, double rope_base,
+                    void* workspace, size_t workspace_bytes, swa_stream_t stream) {
+  if (!rope_base_ok(rope_base)) return SWA_ERR_INVALID_ARG;
+  swa::RopeTable rt;
+  swa::make_rope_table(rope_base, d, &rt);
+  return run_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
+                    scale, workspace, workspace_bytes, &rt, stream);
+}
+
+int swa_rope_qk(void* q, void* k, const int32_t* positions, long long n_tokens, int Hq, int Hkv, int d,
+                double rope_base, swa_stream_t stream) {
+  if (n_tokens < 0 || Hq < 0 || (k != nullptr && Hkv < 0) || !rope_base_ok(rope_base))
+    return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  if (n_tokens == 0 || (Hq == 0 && (k == nullptr || Hkv == 0))) return SWA_OK;
+  if (!positions || (reinterpret_cast<uintptr_t>(positions) & 3u) || (Hq > 0 && (!q || !aligned16(q))) ||
+      (k != nullptr && !aligned16(k)))
+    return SWA_ERR_INVALID_ARG;
+  swa::RopeTable rt;
+  swa::make_rope_table(rope_base, d, &rt);
+  cudaError_t e = swa::launch_rope_qk(Hq > 0 ? q : nullptr, k, positions, n_tokens, Hq, k ? Hkv : 0, d, rt,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_rope_cache_append(const void* k_new, const void* v_new, const int32_t* pos, void* kcache,
+                          void* vcache, void* sink_k, void* sink_v, int B, int Hkv, int d, int window,
+                          int n_sink, double rope_base, swa_stream_t stream) {
+  if (!rope_base_ok(rope_base)) return SWA_ERR_INVALID_ARG;
+  int st = check_cache(B, Hkv, d, window, n_sink, kcache, vcache, sink_k, sink_v);
+  if (st != SWA_OK) return st;
+  if (B == 0) return SWA_OK;
+  if (!k_new || !v_new || !pos || !aligned16(k_new) || !aligned16(v_new) ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  swa::RopeTable rt;
+  swa::make_rope_table(rope_base, d, &rt);
+  cudaError_t e = swa::launch_rope_append(k_new, v_new, pos, kcache, vcache, sink_k, sink_v, B, Hkv, d,
+                                          window, n_sink, rt, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

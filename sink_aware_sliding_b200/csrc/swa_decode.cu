@@ -28,6 +28,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "rope.cuh"
 #include "swa_internal.h"
 
 namespace swa {
@@ -94,9 +95,9 @@ struct Block {
   uint4 v[4][DCfg<D>::VCH];   // keys 2t, 2t+1, 2t+8, 2t+9
 };
 
-template <int D>
+template <int D, bool ROPE>
 __global__ void __launch_bounds__(kDecodeThreads)
-    swa_decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+    swa_decode_split_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ RopeTable rt) {
   using C = DCfg<D>;
   extern __shared__ long long s_pre[];  // B + 1
   const int lane = threadIdx.x & 31;
@@ -153,11 +154,20 @@ __global__ void __launch_bounds__(kDecodeThreads)
       const bool real = g < G;
       const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) +
                                   (static_cast<size_t>(b) * a.Hq + kvh * G + (real ? g : 0)) * D;
+      uint4 w[C::KCH];
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c)
+        w[c] = real ? *reinterpret_cast<const uint4*>(qrow + c * 32 + t * 8) : make_uint4(0, 0, 0, 0);
+      if constexpr (ROPE) {
+        // rotate-half partner of element c*32 + t*8 + e is in chunk c + KCH/2 of the same thread
+        if (real)
+#pragma unroll
+          for (int c = 0; c < C::KCH / 2; ++c) rope_rotate_chunks(w[c], w[c + C::KCH / 2], p, c * 32 + t * 8, rt.theta);
+      }
 #pragma unroll
       for (int c = 0; c < C::KCH; ++c) {
-        uint4 w = real ? *reinterpret_cast<const uint4*>(qrow + c * 32 + t * 8) : make_uint4(0, 0, 0, 0);
-        qa[2 * c][0] = w.x; qa[2 * c][1] = w.y;
-        qa[2 * c + 1][0] = w.z; qa[2 * c + 1][1] = w.w;
+        qa[2 * c][0] = w[c].x; qa[2 * c][1] = w[c].y;
+        qa[2 * c + 1][0] = w[c].z; qa[2 * c + 1][1] = w[c].w;
       }
     }
     float o[C::MT][4];
@@ -334,9 +344,15 @@ __global__ void __launch_bounds__(128) swa_decode_merge_kernel(const __grid_cons
 }
 
 template <int D>
-cudaError_t launch_decode_impl(const DecodeArgs& a, int grid, int block, cudaStream_t stream) {
+cudaError_t launch_decode_impl(const DecodeArgs& a, int grid, int block, cudaStream_t stream,
+                               const RopeTable* rope) {
   const size_t smem = sizeof(long long) * (a.B + 1);
-  swa_decode_split_kernel<D><<<grid, block, smem, stream>>>(a);
+  if (rope != nullptr) {
+    swa_decode_split_kernel<D, true><<<grid, block, smem, stream>>>(a, *rope);
+  } else {
+    const RopeTable unused{};
+    swa_decode_split_kernel<D, false><<<grid, block, smem, stream>>>(a, unused);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   swa_decode_merge_kernel<D><<<a.B * a.Hkv, 128, 0, stream>>>(a);
@@ -404,18 +420,19 @@ __global__ void swa_cache_append_kernel(const uint4* __restrict__ k, const uint4
 
 size_t decode_partial_floats(int G, int d) { return static_cast<size_t>(G) * (d + 2); }
 
-cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream) {
-  if (d == 128) return launch_decode_impl<128>(a, grid, block, stream);
-  if (d == 64) return launch_decode_impl<64>(a, grid, block, stream);
+cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream,
+                          const RopeTable* rope) {
+  if (d == 128) return launch_decode_impl<128>(a, grid, block, stream, rope);
+  if (d == 64) return launch_decode_impl<64>(a, grid, block, stream, rope);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t decode_occupancy(int d, int B, int* ctas_per_sm) {
   const size_t smem = sizeof(long long) * (B + 1);
   if (d == 128)
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, swa_decode_split_kernel<128>,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, swa_decode_split_kernel<128, false>,
                                                          kDecodeThreads, smem);
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, swa_decode_split_kernel<64>,
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, swa_decode_split_kernel<64, false>,
                                                        kDecodeThreads, smem);
 }
 

@@ -52,14 +52,6 @@ struct HadCfg {
   static constexpr int R = TB - P2;                       // bits done in pass 3
   static constexpr int CTA = NT >= 256 ? NT : 256;        // threads per CTA
   static constexpr int ROWS = CTA / NT;                   // rows per CTA
-  // pass 3 works on quads (4 consecutive elements) x 2^R; a row has GPR such
-  // groups, covered by GW threads; the CTA's threads form TEAMS teams and each
-  // thread applies one load of its alpha/beta to RPT rows
-  static constexpr int GPR = TB > 0 ? N / (4 << (TB - (TB < 5 ? TB : 5))) : 1;
-  static constexpr int GW = GPR < CTA ? GPR : CTA;
-  static constexpr int TEAMS = CTA / GW;
-  static constexpr int GQ = GPR / GW;
-  static constexpr int RPT = ROWS / TEAMS;
   // padded fp32 row in shared memory (floats), a multiple of 4
   static constexpr int XROW = TB > 0 ? ((N + N / 8 + ((8 * N) >> (3 + P2)) + 3) / 4) * 4 : 0;
   static constexpr size_t SMEM = sizeof(float) * ROWS * XROW;
@@ -224,12 +216,19 @@ __global__ void __launch_bounds__(HadCfg<LOGN>::CTA)
 
     // pass 3: the remaining R bits on quads of consecutive elements; thread tau
     // takes quad groups lg, lg + GW, ... of rows team, team + TEAMS, ...
+    // a row has GPR quad groups, covered by GW threads; the CTA's threads form
+    // TEAMS teams and each thread applies one load of its alpha/beta to RPT rows
     constexpr int M3 = 1 << R;
-    const int team = static_cast<int>(threadIdx.x) / Cfg::GW, lg = static_cast<int>(threadIdx.x) % Cfg::GW;
+    constexpr int GPR = N / (4 * M3);
+    constexpr int GW = GPR < Cfg::CTA ? GPR : Cfg::CTA;
+    constexpr int TEAMS = Cfg::CTA / GW;
+    constexpr int GQ = GPR / GW;
+    constexpr int RPT = ROWS / TEAMS;
+    const int team = static_cast<int>(threadIdx.x) / GW, lg = static_cast<int>(threadIdx.x) % GW;
     const long long row0 = static_cast<long long>(blockIdx.x) * ROWS;
 #pragma unroll
-    for (int k = 0; k < Cfg::GQ; ++k) {
-      const int g = lg + k * Cfg::GW;
+    for (int k = 0; k < GQ; ++k) {
+      const int g = lg + k * GW;
       const int base = ((g & 1) << 2) | (((g >> 1) & ((1 << P2) - 1)) << 3) | ((g >> (1 + P2)) << (3 + TB));
       uint64_t av[M3][2], bv[M3][2];
 #pragma unroll
@@ -238,8 +237,8 @@ __global__ void __launch_bounds__(HadCfg<LOGN>::CTA)
         load_pairs4(beta + base + (w << (3 + P2)), bv[w]);
       }
 #pragma unroll 1
-      for (int m = 0; m < Cfg::RPT; ++m) {
-        const int r = team + m * Cfg::TEAMS;
+      for (int m = 0; m < RPT; ++m) {
+        const int r = team + m * TEAMS;
         if (row0 + r >= n_rows) break;                    // rows of a team ascend
         const float* rb = xs + r * Cfg::XROW;
         uint64_t c[2][M3];                                // c[q][w]: pair q of quad w

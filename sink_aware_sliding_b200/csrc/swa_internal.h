@@ -57,7 +57,16 @@ struct DecodeArgs {
   int n_warps;          // total warps of the split kernel
 };
 
-cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream);
+// Rotary frequencies theta_i = base^(-2i/d), i < d/2 (d <= 128), for the fused
+// rotary encoding.
+struct RopeTable {
+  double theta[64];
+};
+void make_rope_table(double base, int d, RopeTable* t);
+
+// rope == nullptr: q is used as given; otherwise q is rotated at pos[b] first.
+cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream,
+                          const RopeTable* rope = nullptr);
 size_t decode_partial_floats(int G, int d);
 cudaError_t decode_occupancy(int d, int B, int* ctas_per_sm);
 int decode_threads();
@@ -67,6 +76,14 @@ cudaError_t launch_cache_fill(const void* k, const void* v, int P, void* kc, voi
 cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* pos, void* kc,
                                 void* vc, void* sk, void* sv, int B, int Hkv, int d, int W, int S,
                                 cudaStream_t stream);
+
+// Rotary encoding in place: q [T, Hq, d], k [T, Hkv, d] (k may be null), token t
+// at positions[t]; and the fused rotate-k-then-append of one decode step.
+cudaError_t launch_rope_qk(void* q, void* k, const int32_t* positions, long long T, int Hq, int Hkv,
+                           int d, const RopeTable& rt, cudaStream_t stream);
+cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, void* kc, void* vc,
+                               void* sk, void* sv, int B, int Hkv, int d, int W, int S,
+                               const RopeTable& rt, cudaStream_t stream);
 
 // Hadamard output projection z = alpha * (y H) + beta over rows of n = 2^k elements.
 struct HadamardArgs {

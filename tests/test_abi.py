@@ -68,3 +68,24 @@ def test_argument_checks_happen_before_any_device_work(lib):
     assert lib.swa_decode_workspace_bytes(1, 12, 1, 128, 64, 4) == 0    # G = 12 > 8
     assert lib.swa_decode_workspace_bytes(1, 4, 3, 128, 64, 4) == 0     # Hq % Hkv != 0
     assert lib.swa_decode_workspace_bytes(1, 4, 1, 80, 64, 4) == 0      # d = 80
+
+
+def test_rope_and_hadamard_argument_checks(lib):
+    D = ctypes.c_double
+    # rotary encoding: the base and d are checked first, then empty work returns OK
+    assert lib.swa_rope_qk(None, None, None, 10, 4, 2, 128, D(0.0), None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_rope_qk(None, None, None, 10, 4, 2, 128, D(float("nan")), None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_rope_qk(None, None, None, -1, 4, 2, 128, D(1e4), None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_rope_qk(None, None, None, 10, 4, 2, 96, D(1e4), None) == swa.SWA_ERR_UNSUPPORTED
+    assert lib.swa_rope_qk(None, None, None, 0, 4, 2, 128, D(1e4), None) == swa.SWA_OK
+    assert lib.swa_rope_qk(None, None, None, 10, 4, 2, 128, D(1e4), None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_rope_cache_append(None, None, None, None, None, None, None, 1, 2, 128, 64, 4,
+                                     D(-1.0), None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_decode_rope(None, None, None, None, None, None, None, None, 1, 4, 2, 128, 64, 4,
+                               ctypes.c_float(0.1), D(float("inf")), None, 0, None) == swa.SWA_ERR_INVALID_ARG
+    # Hadamard projection: n must be a power of two in [32, 8192]
+    for n in (16, 48, 16384):
+        assert lib.swa_hadamard_proj(None, None, None, None, 4, n, 0, None) == swa.SWA_ERR_UNSUPPORTED
+    assert lib.swa_hadamard_proj(None, None, None, None, 4, 64, 2, None) == swa.SWA_ERR_INVALID_ARG
+    assert lib.swa_hadamard_proj(None, None, None, None, 0, 64, 0, None) == swa.SWA_OK
+    assert lib.swa_hadamard_proj(None, None, None, None, 4, 64, 0, None) == swa.SWA_ERR_INVALID_ARG
