@@ -10,8 +10,9 @@ L=2048, d=64, window 128), counting 4*d FLOPs per visible (query, key) pair.
 The same line carries, under "workloads", the other workloads measured the
 same way: the 8B-shaped GQA prefill and the packed long-context prefill
 (TFLOP/s against the tensor roofline) and the ring-buffer decode (HBM GB/s and
-tokens/s against the HBM roofline) and the Hadamard output projection of the
-GQA prefill's output (HBM GB/s).
+tokens/s against the HBM roofline), the same decode with the rotary encoding
+fused into append and decode, the rotary encoding of the GQA prefill's q and k,
+and the Hadamard output projection of the GQA prefill's output (HBM GB/s).
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -407,6 +408,77 @@ def bench_hadamard(name, steps, warmup, dev, flush, peaks, sampler):
     }
 
 
+def bench_rope_qk(name, steps, warmup, dev, flush, peaks, sampler):
+    """Rotary encoding of a prefill's q and k in place (HBM-bound: read and write both)."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    c = wl.ROPE_WORKLOADS[name]
+    T, Hq, Hkv, d, base = c["T"], c["Hq"], c["Hkv"], c["d"], c["rope_base"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.SEED)
+    q = torch.randn(T, Hq, d, generator=g, device=dev).bfloat16()
+    k = torch.randn(T, Hkv, d, generator=g, device=dev).bfloat16()
+    pos = torch.arange(T, dtype=torch.int32, device=dev)
+
+    def run(qq=q, kk=k):
+        swa.swa_rope_qk(qq, kk, pos, base)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    alg_bytes = 2 * T * (Hq + Hkv) * d * 2 + 4 * T
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+
+    hq, hk = q.cpu().pin_memory(), k.cpu().pin_memory()
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        run(dq, dk)
+        hq.copy_(dq, non_blocking=True)
+        hk.copy_(dk, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(3, steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    nb = (q.numel() + k.numel()) * 2
+    roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "traffic": profiled_traffic(name), "algorithmic_bytes_per_launch": alg_bytes}
+    return {
+        "config": {"workload": name, "kind": "rope_qk", "T": T, "Hq": Hq, "Hkv": Hkv, "d": d,
+                   "rope_base": base, "dtype": "bf16"},
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5), "roofline": roof,
+        "e2e": {"value": round(alg_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
 def bench_decode(name, steps, warmup, dev, peaks, sampler):
     """One step = one generated token for all B sequences: cache append + split-K decode + merge."""
     import torch
@@ -420,6 +492,9 @@ def bench_decode(name, steps, warmup, dev, peaks, sampler):
     z = dict(device=dev, dtype=torch.bfloat16)
     kc, vc = torch.empty(B, Hkv, W, d, **z), torch.empty(B, Hkv, W, d, **z)
     sk, sv = torch.empty(B, Hkv, S, d, **z), torch.empty(B, Hkv, S, d, **z)
+    if w.rope_base > 0:                # the prefix keys enter the cache rotated
+        pp = torch.arange(w.prefix, dtype=torch.int32, device=dev).repeat(B)
+        swa.swa_rope_qk(di.prefix_k, None, pp, w.rope_base)
     swa.swa_cache_fill(di.prefix_k, di.prefix_v, kc, vc, sk, sv, W, S)
     del di.prefix_k, di.prefix_v
     pos = torch.arange(w.prefix, w.prefix + n_tok + warmup, dtype=torch.int32, device=dev)
@@ -428,9 +503,23 @@ def bench_decode(name, steps, warmup, dev, peaks, sampler):
     lse = torch.empty(B, Hq, device=dev, dtype=torch.float32)
     ws = torch.empty(swa.swa_decode_workspace_bytes(B, Hq, Hkv, d, W, S), device=dev, dtype=torch.uint8)
 
+    rope = w.rope_base > 0
+
+    def append(kn, vn, p):
+        if rope:
+            swa.swa_rope_cache_append(kn, vn, p, kc, vc, sk, sv, W, S, w.rope_base)
+        else:
+            swa.swa_cache_append(kn, vn, p, kc, vc, sk, sv, W, S)
+
+    def dec(qq, p):
+        if rope:
+            swa.swa_decode_rope(qq, kc, vc, sk, sv, p, out, lse, W, S, ws, w.rope_base)
+        else:
+            swa.swa_decode(qq, kc, vc, sk, sv, p, out, lse, W, S, ws)
+
     def step(i):
-        swa.swa_cache_append(di.k_new[i], di.v_new[i], pos[i], kc, vc, sk, sv, W, S)
-        swa.swa_decode(di.q[i], kc, vc, sk, sv, pos[i], out, lse, W, S, ws)
+        append(di.k_new[i], di.v_new[i], pos[i])
+        dec(di.q[i], pos[i])
 
     for i in range(warmup):
         step(i)
@@ -449,7 +538,7 @@ def bench_decode(name, steps, warmup, dev, peaks, sampler):
     # dominant kernel (split-K decode + merge) timed per call on the same stream
     timer = Timer(torch)
     for i in range(warmup, warmup + min(n_tok, 64)):
-        timer(lambda i=i: swa.swa_decode(di.q[i], kc, vc, sk, sv, pos[i], out, lse, W, S, ws))
+        timer(lambda i=i: dec(di.q[i], pos[i]))
     dec_ms = statistics.mean(timer.ms())
     p_last = w.prefix + warmup + n_tok - 1
     step_bytes = decode_step_bytes(w, p_last)
@@ -470,8 +559,8 @@ def bench_decode(name, steps, warmup, dev, peaks, sampler):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dp.copy_(hp, non_blocking=True)
-        swa.swa_cache_append(dk, dv, dp, kc, vc, sk, sv, W, S)
-        swa.swa_decode(dq, kc, vc, sk, sv, dp, out, lse, W, S, ws)
+        append(dk, dv, dp)
+        dec(dq, dp)
         ho.copy_(out, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -575,6 +664,16 @@ def profile_case(args):
             swa.swa_hadamard_proj(y, alpha, beta, z)
         torch.cuda.synchronize()
         return
+    if args.profile_case in wl.ROPE_WORKLOADS:
+        c = wl.ROPE_WORKLOADS[args.profile_case]
+        T = args.L or c["T"]
+        q = torch.randn(T, c["Hq"], c["d"], device=dev).bfloat16()
+        k = torch.randn(T, c["Hkv"], c["d"], device=dev).bfloat16()
+        pos = torch.arange(T, dtype=torch.int32, device=dev)
+        for _ in range(n):
+            swa.swa_rope_qk(q, k, pos, c["rope_base"])
+        torch.cuda.synchronize()
+        return
     w = wl.WORKLOADS[args.profile_case]
     if w.kind == "prefill":
         q, k, v = wl.make_prefill(w, device=dev, B=args.B, L=args.L)
@@ -602,8 +701,14 @@ def profile_case(args):
                          device=dev, dtype=torch.uint8)
         for i in range(n):
             pos = torch.full((B,), w.prefix + i, dtype=torch.int32, device=dev)
-            swa.swa_cache_append(di.k_new[i], di.v_new[i], pos, kc, vc, sk, sv, w.window, w.n_sink)
-            swa.swa_decode(di.q[i], kc, vc, sk, sv, pos, out, lse, w.window, w.n_sink, ws)
+            if w.rope_base > 0:
+                swa.swa_rope_cache_append(di.k_new[i], di.v_new[i], pos, kc, vc, sk, sv, w.window,
+                                          w.n_sink, w.rope_base)
+                swa.swa_decode_rope(di.q[i], kc, vc, sk, sv, pos, out, lse, w.window, w.n_sink, ws,
+                                    w.rope_base)
+            else:
+                swa.swa_cache_append(di.k_new[i], di.v_new[i], pos, kc, vc, sk, sv, w.window, w.n_sink)
+                swa.swa_decode(di.q[i], kc, vc, sk, sv, pos, out, lse, w.window, w.n_sink, ws)
     torch.cuda.synchronize()
     if swa.swa_device_error() != 0:
         raise SystemExit("device wait timed out")
@@ -616,7 +721,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
-    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,hadamard_proj")
+    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -662,8 +767,10 @@ def main():
         names.insert(0, HEADLINE)
     results = {}
     for n in names:
-        if n == "decode":
+        if n in ("decode", "decode_rope"):
             results[n] = bench_decode(n, args.decode_tokens, args.warmup, dev, peaks, sampler)
+        elif n == "rope_qk_gqa8b":
+            results[n] = bench_rope_qk(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         elif n == "hadamard_proj":
             results[n] = bench_hadamard(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         else:

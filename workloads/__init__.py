@@ -49,6 +49,7 @@ class Workload:
     sink_bias: bool = False
     prefix: int = 0                # decode: tokens already in context
     steps: int = 0                 # decode: generated tokens
+    rope_base: float = 0.0         # > 0: rotary encoding applied on the device (decode steps)
     note: str = ""
 
     @property
@@ -69,6 +70,8 @@ class Workload:
             out.update(seqlens=list(self.seqlens))
         else:
             out.update(B=self.B, prefix=self.prefix, steps=self.steps)
+        if self.rope_base > 0:
+            out.update(rope_base=self.rope_base)
         return out
 
 
@@ -86,6 +89,10 @@ WORKLOADS = {
         "decode", "decode", Hq=32, Hkv=8, d=128, window=4096, n_sink=4, dtype="bf16",
         B=64, prefix=16384, steps=1024, sink_bias=True,
         note="ring-buffer decode after a 16384-token prefix"),
+    "decode_rope": Workload(
+        "decode_rope", "decode", Hq=32, Hkv=8, d=128, window=4096, n_sink=4, dtype="bf16",
+        B=64, prefix=16384, steps=1024, sink_bias=True, rope_base=10000.0,
+        note="the decode workload with the rotary encoding fused into append and decode"),
     "packed_long": Workload(
         "packed_long", "varlen", Hq=32, Hkv=8, d=128, window=2048, n_sink=4, dtype="bf16",
         seqlens=(131072, 65536, 16384, 1000), note="four packed sequences"),
@@ -247,6 +254,11 @@ class ProjWorkload:
         return {"workload": self.name, "kind": "hadamard_proj", "T": self.T, "n": self.n,
                 "in_dtype": "bf16", "out_dtype": self.out_dtype}
 
+
+ROPE_WORKLOADS = {
+    # rotary encoding of the 8B-shaped prefill's q and k before attention
+    "rope_qk_gqa8b": dict(T=32768, Hq=32, Hkv=8, d=128, rope_base=10000.0),
+}
 
 PROJ_WORKLOADS = {
     "hadamard_proj": ProjWorkload(
