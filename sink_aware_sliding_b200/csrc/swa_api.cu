@@ -138,7 +138,13 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
     units = (T / swa::kBM + n_seq) * static_cast<long long>(Hq);  // upper bound
     if (units > INT32_MAX) return SWA_ERR_UNSUPPORTED;
   }
-  // Debug flag 2 forces the one-tile kernel (so tests can check both kernels).
+  // Debug flag 4 skips the short-window stream kernel, flag 2 forces the one-tile
+  // kernel (so tests can check every kernel on the same inputs).
+  if ((a.debug_flags & 6) == 0 && swa::prefill_stream_supported(d, f32, window, n_sink)) {
+    const int grid_s = static_cast<int>(std::min<long long>(dev->sms, units));
+    cudaError_t es = swa::launch_prefill_stream(a, tq, tk, tv, to, dtype != SWA_DTYPE_BF16, grid_s, stream);
+    if (es != cudaErrorNotSupported) return es == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+  }
   const bool pair = (a.debug_flags & 2) == 0 && swa::prefill_pair_supported(Hq, Hq / Hkv, d, f32);
   if (pair) units = (units + 1) / 2;
   const int grid = static_cast<int>(std::min<long long>(dev->sms, units));

@@ -36,6 +36,11 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
 
 // Two-query-tile prefill (heads 2p, 2p+1 per CTA); used when Hq is even and the
 // ring can hold two key tiles (always for 16 KB tiles, else when pairs share a KV head).
+// Short-window stream kernel: d = 64, bf16 inputs, window <= 129, no sink prefix.
+bool prefill_stream_supported(int d, bool f32, int window, int n_sink);
+cudaError_t launch_prefill_stream(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const CUtensorMap& to, bool out_f32, int grid,
+                                  cudaStream_t stream);
 bool prefill_pair_supported(int Hq, int G, int d, bool f32);
 // `to` maps the output (bf16, same box as q); it is used for d = 64 bf16 output only.
 cudaError_t launch_prefill_pair(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
