@@ -244,9 +244,10 @@ unsigned long long swa_set_wait_timeout_ns(unsigned long long ns);
 /*
  * Test hooks, process-wide.  Bit 0 makes the prefill kernels' load warp issue
  * no copies, so that its consumers' bounded waits run out; bit 1 makes
- * swa_fwd / swa_fwd_varlen use the one-query-tile kernel even where the
- * two-tile kernel applies.  0 restores normal operation.  Returns the
- * previous flags.
+ * swa_fwd / swa_fwd_varlen use the one-query-tile kernel even where another
+ * kernel applies; bit 2 keeps them off the short-window stream kernel (d = 64,
+ * window <= 129, no sinks), so the two-tile kernel runs instead.  0 restores
+ * normal operation.  Returns the previous flags.
  */
 int swa_set_debug_flags(int flags);
 
