@@ -296,3 +296,46 @@ def rope(x, positions, base: float = 10000.0) -> np.ndarray:
     c, s = np.cos(ang).reshape(shape), np.sin(ang).reshape(shape)
     lo, hi = x[..., : d // 2], x[..., d // 2:]
     return np.concatenate([lo * c - hi * s, lo * s + hi * c], axis=-1)
+
+
+# ---------------------------------------------------------------------------
+# Backward pass of sink-aware sliding-window attention: gradients of the loss
+# with respect to q, k and v given dO = dL/dout, for the visible set of
+# "Sliding-window beats linear attention" (sections 1 and 3).  Written out from
+# the definition P = softmax over the visible keys, out = P V:
+#     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
+#     dQ = scale * dS K,  dK = scale * dS^T Q,
+# the gradients of a KV head summed over the query heads that read it.
+# Dense per (sequence, head) in float64; sizes up to a few thousand rows.
+# ---------------------------------------------------------------------------
+
+def visible_mask(L: int, window: int, n_sink: int) -> np.ndarray:
+    """Boolean [L, L]: row t sees key j iff j <= t and (j >= t - window + 1 or j < n_sink)."""
+    t = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    return (j <= t) & ((j >= t - window + 1) | (j < n_sink))
+
+
+def swa_bwd(q, k, v, dout, window: int, n_sink: int, scale: float):
+    """q, dout [B, L, Hq, d]; k, v [B, L, Hkv, d] -> dq, dk, dv (float64, same shapes)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    M = visible_mask(L, window, n_sink)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            kh = h // G
+            s = scale * (q[b, :, h] @ k[b, :, kh].T)
+            s = np.where(M, s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            dp = do[b, :, h] @ v[b, :, kh].T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dq[b, :, h] = scale * (ds @ k[b, :, kh])
+            dk[b, :, kh] += scale * (ds.T @ q[b, :, h])
+            dv[b, :, kh] += p.T @ do[b, :, h]
+    return dq, dk, dv
