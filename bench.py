@@ -12,7 +12,8 @@ same way: the 8B-shaped GQA prefill and the packed long-context prefill
 (TFLOP/s against the tensor roofline) and the ring-buffer decode (HBM GB/s and
 tokens/s against the HBM roofline), the same decode with the rotary encoding
 fused into append and decode, the rotary encoding of the GQA prefill's q and k,
-and the Hadamard output projection of the GQA prefill's output (HBM GB/s).
+the Hadamard output projection of the GQA prefill's output (HBM GB/s), and the
+backward pass of the Based-shaped and (at L=8192) the 8B-shaped prefill.
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -479,6 +480,56 @@ def bench_rope_qk(name, steps, warmup, dev, flush, peaks, sampler):
     }
 
 
+def bench_bwd(name, steps, warmup, dev, flush, peaks, sampler):
+    """Backward pass (dq, dk, dv) of a prefill workload; FLOPs: five products of 2*d per
+    visible pair and query head (S, dP, dV, dK, dQ), i.e. 2.5x the forward's."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    fwd_name, L = wl.BWD_WORKLOADS[name]
+    w = wl.WORKLOADS[fwd_name]
+    q, k, v = wl.make_prefill(w, device=dev, L=L)
+    B, Lr = q.shape[0], q.shape[1]
+    out = torch.empty_like(q)
+    lse = torch.empty(B, w.Hq, Lr, device=dev, dtype=torch.float32)
+    swa.swa_fwd(q, k, v, out, lse, w.window, w.n_sink)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.SEED + 1)
+    do = torch.randn(q.shape, generator=g, device=dev).bfloat16()
+    dq = torch.empty(q.shape, device=dev)
+    dk = torch.empty(k.shape, device=dev)
+    dv = torch.empty_like(dk)
+
+    def run():
+        swa.swa_bwd(q, k, v, out, do, lse, dq, dk, dv, w.window, w.n_sink)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    if swa.swa_device_error() != 0:
+        raise RuntimeError(f"{name}: device wait timed out")
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    flops = 2.5 * prefill_flops(w, [Lr] * B)
+    tflops = flops / (ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tflops / peaks["bf16_tflops"], 4), "peak_source": peaks["source"],
+            "flops_per_launch": flops, "traffic": None}
+    cfg = dict(w.describe(), L=Lr, workload=name, **{"pass": "backward"})
+    return {"config": cfg, "value": round(tflops, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "roofline": roof, "gpu_launches": 2 * steps, "l2": "flushed between steps (512 MiB write)"}
+
+
 def bench_decode(name, steps, warmup, dev, peaks, sampler):
     """One step = one generated token for all B sequences: cache append + split-K decode + merge."""
     import torch
@@ -721,7 +772,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
-    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj")
+    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj,"
+                    "bwd_based_local,bwd_gqa8b_L8192")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -769,6 +821,8 @@ def main():
     for n in names:
         if n in ("decode", "decode_rope"):
             results[n] = bench_decode(n, args.decode_tokens, args.warmup, dev, peaks, sampler)
+        elif n.startswith("bwd_"):
+            results[n] = bench_bwd(n, max(3, args.steps // 4), args.warmup, dev, flush, peaks, sampler)
         elif n == "rope_qk_gqa8b":
             results[n] = bench_rope_qk(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         elif n == "hadamard_proj":

@@ -166,6 +166,23 @@ int swa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                        swa_stream_t stream);
 
 /*
+ * Backward pass of sink-aware sliding-window attention (the gradients of the
+ * forward above; visible set of "Sliding-window beats linear attention",
+ * sections 1 and 3).  With P the forward's weights (recomputed from lse) and
+ * D_t = rowsum(dout_t * out_t):
+ *   dv = P^T dout,  dS = P * (dout v^T - D),  dq = scale dS k,  dk = scale dS^T q,
+ * the gradients of a KV head summed over the query heads that read it.
+ *   q, out, dout [B, L, Hq, d] bf16;  k, v [B, L, Hkv, d] bf16   (read)
+ *   lse [B, Hq, L] float32: the forward's log-sum-exp                (read)
+ *   dq [B, L, Hq, d], dk, dv [B, L, Hkv, d] float32                   (written)
+ * Supported: d = 64 or 128, fixed-length batches.  Arguments and errors as
+ * swa_fwd; a bounded device wait that runs out sets SWA_ERR_DEVICE_TIMEOUT.
+ */
+int swa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+            float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int L, int d, int window, int n_sink,
+            float scale, swa_stream_t stream);
+
+/*
  * Rotary position encoding of the sliding-window branch ("Simple linear
  * attention language models balance the recall-throughput tradeoff", proposed
  * method: the window attention uses rotary position encoding, the linear branch

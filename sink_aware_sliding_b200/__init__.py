@@ -36,7 +36,7 @@ EXPORTS = (
     "swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append",
     "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
-    "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope",
+    "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope", "swa_bwd",
 )
 
 _lib = None
@@ -69,6 +69,7 @@ def _load():
     lib.swa_rope_qk.argtypes = [P, P, P, LL, I, I, I, D, P]
     lib.swa_rope_cache_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P]
     lib.swa_decode_rope.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, D, P, SZ, P]
+    lib.swa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
@@ -77,7 +78,7 @@ def _load():
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
-                 "swa_decode_rope",
+                 "swa_decode_rope", "swa_bwd",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -250,6 +251,21 @@ def swa_decode_noalloc(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window:
                                     _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window),
                                     int(n_sink), _scale(scale, d), _stream(stream))
     _check(st, "swa_decode_noalloc")
+
+
+def swa_bwd(q, k, v, out, dout, lse, dq, dk, dv, window: int, n_sink: int, scale=None, stream=None) -> None:
+    """Gradients dq [B, L, Hq, d], dk, dv [B, L, Hkv, d] (float32) of the forward
+    out = swa_fwd(q, k, v), given dout (bf16) and the forward's out (bf16) and lse."""
+    import torch
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t.dtype == torch.bfloat16 and t.is_contiguous(), f"{name} bf16 contiguous")
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (lse, "lse")):
+        _need(t.dtype == torch.float32 and t.is_contiguous(), f"{name} float32 contiguous")
+    st = _load().swa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                         _ptr(dv), B, Hq, Hkv, L, d, int(window), int(n_sink), _scale(scale, d), _stream(stream))
+    _check(st, "swa_bwd")
 
 
 def swa_hadamard_proj(y, alpha, beta, z, stream=None) -> None:

@@ -363,6 +363,52 @@ int swa_rope_cache_append(const void* k_new, const void* v_new, const int32_t* p
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+int swa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+            float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int L, int d, int window, int n_sink,
+            float scale, swa_stream_t stream) {
+  int st = check_heads(Hq, Hkv, d, window, n_sink, scale, SWA_DTYPE_BF16);
+  if (st != SWA_OK) return st;
+  if (B < 0 || L < 0) return SWA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * L == 0) return SWA_OK;
+  const void* ptrs[9] = {q, k, v, out, dout, dq, dk, dv, nullptr};
+  for (int i = 0; i < 8; ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return SWA_ERR_INVALID_ARG;
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_INVALID_ARG;
+  const long long T = static_cast<long long>(B) * L;
+  if (T > INT32_MAX || T * Hq > INT32_MAX) return SWA_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != SWA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((st = make_map(&tq, q, false, d, Hq, T, swa::kBM)) != SWA_OK) return st;
+  if ((st = make_map(&tk, k, false, d, Hkv, T, swa::kBN)) != SWA_OK) return st;
+  if ((st = make_map(&tv, v, false, d, Hkv, T, swa::kBN)) != SWA_OK) return st;
+  if ((st = make_map(&tdo, dout, false, d, Hq, T, swa::kBM)) != SWA_OK) return st;
+  swa::BwdArgs ba{};
+  swa::PrefillArgs& a = ba.pa;
+  a.n_seq = B;
+  a.L = L;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.window = window;
+  a.n_sink = n_sink;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.total_tiles = static_cast<int>(static_cast<long long>(B) * ((L + swa::kBM - 1) / swa::kBM));
+  a.timeout_ns = g_timeout_ns.load();
+  a.debug_flags = g_debug_flags.load();
+  a.err = dev->err;
+  ba.out = out;
+  ba.dout = dout;
+  ba.lse = lse;
+  ba.dq = dq;
+  ba.dk = dk;
+  ba.dv = dv;
+  cudaError_t e = swa::launch_bwd(ba, tq, tk, tv, tdo, d, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 int swa_hadamard_proj(const void* y, const float* alpha, const float* beta, void* z,
                       long long n_rows, int n, int out_dtype, swa_stream_t stream) {
   if (n_rows < 0 || n < 32 || n > 8192 || (n & (n - 1)) != 0) return n_rows < 0 ? SWA_ERR_INVALID_ARG

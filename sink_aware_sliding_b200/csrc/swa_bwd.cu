@@ -1,0 +1,482 @@
+// Backward pass of sink-aware sliding-window attention, sm_100a (d = 64 or 128,
+// bf16 inputs, fp32 gradients).  The visible set is the forward's ("Sliding-window
+// beats linear attention", sections 1 and 3): row t sees key j iff j <= t and
+// (j >= t - window + 1 or j < n_sink).  With P the forward's softmax (recomputed
+// from the saved log-sum-exp) and D_t = rowsum(dO_t * O_t):
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Two kernels, neither needing atomics:
+//   swa_bwd_dkdv_kernel  one CTA per (sequence, KV head, 128-key tile): for every
+//                        query head of that KV head and every query tile that sees
+//                        the key tile (the band, or all later tiles for a tile
+//                        holding sinks) it computes S^T = K Q^T and dP^T = V dO^T on
+//                        tcgen05, forms P^T and dS^T per key row (thread = TMEM lane =
+//                        key), and accumulates dV += P^T dO and dK += dS^T Q in TMEM;
+//   swa_bwd_dq_kernel    one CTA per (sequence, query head, 128-row query tile): for
+//                        the key tiles the forward visits it computes S and dP, forms
+//                        dS per query row and accumulates dQ += dS K in TMEM.
+// Each CTA is one warpgroup; thread 0 issues TMA and MMA, all threads do the
+// element-wise step; every hand-off is an mbarrier with a bounded wait.  Thread 0
+// shares warp 0 with element-wise threads, so the warp is reconverged
+// (__syncwarp) after every issuer-only block and every wait's outcome is made
+// warp-uniform before the warp-collective tcgen05 instructions that follow.  This is
+// the first, non-overlapped version: loads, products and the element-wise step of
+// one tile pair run one after another.
+//
+// TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
+// written over their first halves), dV 256.., dK 256+d..; (dQ kernel): S 0-127,
+// dP 128-255, dQ 256...
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "prefill_common.cuh"
+
+namespace swa {
+namespace {
+
+using namespace prefill;
+
+constexpr int kBwdThreads = 128;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE = kBM * D * 2;             // one 128-row bf16 tile
+  static constexpr int NCHUNK = D / 64;                // 128-byte column chunks
+  static constexpr int QK_STEPS = D / 16;
+  static constexpr int PV_STEPS = kBN / 16;
+  // shared layout: tiles 0..3, then D_s, L_s (128 floats each), then barriers
+  static constexpr int OFF_T = 0;
+  static constexpr int OFF_DS = 4 * TILE;
+  static constexpr int OFF_LS = OFF_DS + 512;
+  static constexpr int OFF_BAR = OFF_LS + 512;
+  static constexpr int NBAR = 8;
+  static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
+  // Each CTA allocates all 512 TMEM columns, so no second CTA may share the SM
+  // (its allocation would have to wait): ask for more than half of the SM's
+  // shared memory even where the tiles need less.
+  static constexpr int SMEM_USED = OFF_TMEMPTR + 16 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_USED > 119808 ? SMEM_USED : 119808;
+  static constexpr uint32_t IDESC_SS = make_idesc(1u, kBM, kBN, false);   // 128 x 128 scores
+  static constexpr uint32_t IDESC_ACC = make_idesc(1u, kBM, D, true);     // 128 x d accumulators
+};
+
+// barrier indices
+constexpr int kBarA = 0;      // K,V (dK/dV kernel) or Q,dO (dQ kernel): loaded once
+constexpr int kBarB = 1;      // the per-iteration tile pair
+constexpr int kBarS = 2;      // both score products done
+constexpr int kBarP = 3;      // all 128 rows wrote their P / dS (count 128)
+constexpr int kBarO = 4;      // accumulation products done
+constexpr int kBarRow = 5;    // per-iteration row data (D, lse) written (count 128)
+constexpr int kBarDrain = 6;
+
+__device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const PrefillArgs& a) {
+  for (int i = 0; i < 256; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > a.timeout_ns) {
+      atomicCAS(a.err, 0, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// D_t = sum_c dO[t, c] O[t, c] for one row of d bf16 elements (fp32 accumulation).
+template <int D>
+__device__ __forceinline__ float row_dot(const __nv_bfloat16* x, const __nv_bfloat16* y) {
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D; c += 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(x + c);
+    const uint4 w = *reinterpret_cast<const uint4*>(y + c);
+    const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(uu[i] << 16), __uint_as_float(ww[i] << 16), acc);
+      acc = fmaf(__uint_as_float(uu[i] & 0xffff0000u), __uint_as_float(ww[i] & 0xffff0000u), acc);
+    }
+  }
+  return acc;
+}
+
+__device__ __forceinline__ bool visible(int j, int t, const PrefillArgs& a) {
+  return j <= t && t < a.L && (j >= t - a.window + 1 || j < a.n_sink);
+}
+
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int head, int row) {
+#pragma unroll
+  for (int c = 0; c < BwdCfg<D>::NCHUNK; ++c) tma_load_3d(dst + c * (kBM * 128), map, bar, c * 64, head, row);
+}
+
+// ------------------------------------------------------------------ dK, dV
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    swa_bwd_dkdv_kernel(const __grid_constant__ BwdArgs ba, const __grid_constant__ CUtensorMap tq,
+                        const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                        const __grid_constant__ CUtensorMap tdo) {
+  using C = BwdCfg<D>;
+  const PrefillArgs& a = ba.pa;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8 * i; };
+  const uint32_t sK = base + C::OFF_T, sV = sK + C::TILE, sQ = sV + C::TILE, sdO = sQ + C::TILE;
+  float* D_s = reinterpret_cast<float*>(gbase + C::OFF_DS);
+  float* L_s = reinterpret_cast<float*>(gbase + C::OFF_LS);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
+  const int tid = threadIdx.x;
+
+  const int tiles = (a.L + kBM - 1) / kBM;
+  const int jt = blockIdx.x % tiles;
+  const int kvh = (blockIdx.x / tiles) % a.Hkv;
+  const int b = blockIdx.x / (tiles * a.Hkv);
+  const int j0 = jt * kBN;
+  const int it_hi = j0 < a.n_sink ? tiles - 1
+                                  : min(tiles - 1, (min(j0 + kBN - 1, a.L - 1) + a.window - 1) / kBM);
+
+  if (tid == 0) {
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), (i == kBarP || i == kBarRow) ? kBwdThreads : 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (tid < 32) {
+    tmem_alloc(smem_u32(tmem_ptr), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  const uint32_t lane_off = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+  const size_t row_base = static_cast<size_t>(b) * a.L;
+
+  bool ok = true;
+  bool loads_out = false;
+  if (tid == 0) {
+    mbar_expect_tx(bar(kBarA), 2 * C::TILE);
+    load_tile<D>(sK, &tk, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
+    load_tile<D>(sV, &tv, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
+  }
+  int it = 0;
+  const int s_key = j0 + tid;                         // this thread's key (TMEM lane)
+  for (int g = 0; ok && g < a.G; ++g) {
+    const int h = kvh * a.G + g;
+    for (int qi = jt; ok && qi <= it_hi; ++qi, ++it) {
+      const int i0 = qi * kBM;
+      if (tid == 0) {
+        mbar_expect_tx(bar(kBarB), 2 * C::TILE);
+        load_tile<D>(sQ, &tq, bar(kBarB), h, static_cast<int>(row_base) + i0);
+        load_tile<D>(sdO, &tdo, bar(kBarB), h, static_cast<int>(row_base) + i0);
+        loads_out = true;
+      }
+      {  // D and log-sum-exp (log2 units) of query i0 + tid
+        const int t = i0 + tid;
+        float dt = 0.f, l2 = 0.f;
+        if (t < a.L) {
+          const size_t off = ((row_base + t) * a.Hq + h) * D;
+          dt = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + off,
+                          static_cast<const __nv_bfloat16*>(ba.out) + off);
+          l2 = ba.lse[(static_cast<size_t>(b) * a.Hq + h) * a.L + t] * 1.4426950408889634f;
+        }
+        D_s[tid] = dt;
+        L_s[tid] = l2;
+        mbar_arrive(bar(kBarRow));
+      }
+      __syncwarp();
+      if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
+      if (tid == 0) {
+        ok = (it > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB), it & 1, a);
+        if (ok) {
+          loads_out = false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::QK_STEPS; ++kk)
+            umma_ss<false>(tmem, kmajor_desc<4>(sK, kBN, kk), kmajor_desc<4>(sQ, kBM, kk), C::IDESC_SS,
+                           kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < C::QK_STEPS; ++kk)
+            umma_ss<false>(tmem + 128, kmajor_desc<4>(sV, kBN, kk), kmajor_desc<4>(sdO, kBM, kk), C::IDESC_SS,
+                           kk > 0 ? 1u : 0u);
+          tc_commit(bar(kBarS));
+        }
+      }
+      __syncwarp();
+      if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), it & 1, a)))) break;
+      tc_fence_after();
+      // P^T and dS^T of this key row, 64 query columns at a time
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64], dr[64];
+        tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
+        tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
+        tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
+        tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
+        uint32_t pw[32], dw[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float p[2], ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 64 * half + c + e;
+            const bool vis = visible(s_key, i0 + col, a);
+            p[e] = vis ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]) : 0.f;
+            ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
+          }
+          pw[c / 2] = pack_bf16x2(p[0], p[1]);
+          dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st32(tmem + lane_off + 32 * half, pw);
+        tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+      if (tid == 0) {
+        if ((ok = bwd_wait(bar(kBarP), it & 1, a))) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::PV_STEPS; ++kk)
+            umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(sdO, kk), C::IDESC_ACC,
+                           (it == 0 && kk == 0) ? 0u : 1u);
+#pragma unroll
+          for (int kk = 0; kk < C::PV_STEPS; ++kk)
+            umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, v_desc<false, 16>(sQ, kk), C::IDESC_ACC,
+                           (it == 0 && kk == 0) ? 0u : 1u);
+          tc_commit(bar(kBarO));
+        }
+      }
+      __syncwarp();
+      if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
+    }
+  }
+  if (!ok && tid == 0) {
+    // let everything this thread started finish before the CTA releases its memory
+    tc_commit(bar(kBarDrain));
+    bwd_wait(bar(kBarDrain), 0, a);
+    if (it == 0) bwd_wait(bar(kBarA), 0, a);
+    if (loads_out) bwd_wait(bar(kBarB), it & 1, a);
+  }
+  __syncwarp();
+  tc_fence_after();
+  if (__all_sync(0xffffffffu, ok)) {        // warp-uniform: the TMEM loads are warp-collective
+    const bool row_ok = s_key < a.L;
+    float* dv = ba.dv + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
+    float* dk = ba.dk + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t rv[32], rk[32];
+      tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, rv);
+      tmem_ld32_wait(tmem + lane_off + 256 + D + 32 * c, rk);
+      if (!row_ok) continue;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        *reinterpret_cast<float4*>(dv + 32 * c + i) = make_float4(
+            __uint_as_float(rv[i]), __uint_as_float(rv[i + 1]), __uint_as_float(rv[i + 2]), __uint_as_float(rv[i + 3]));
+        *reinterpret_cast<float4*>(dk + 32 * c + i) =
+            make_float4(__uint_as_float(rk[i]) * a.scale, __uint_as_float(rk[i + 1]) * a.scale,
+                        __uint_as_float(rk[i + 2]) * a.scale, __uint_as_float(rk[i + 3]) * a.scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid < 32) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ dQ
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    swa_bwd_dq_kernel(const __grid_constant__ BwdArgs ba, const __grid_constant__ CUtensorMap tq,
+                      const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                      const __grid_constant__ CUtensorMap tdo) {
+  using C = BwdCfg<D>;
+  const PrefillArgs& a = ba.pa;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8 * i; };
+  const uint32_t sQ = base + C::OFF_T, sdO = sQ + C::TILE, sK = sdO + C::TILE, sV = sK + C::TILE;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
+  const int tid = threadIdx.x;
+
+  const int tiles = (a.L + kBM - 1) / kBM;
+  const int qt = blockIdx.x % tiles;
+  const int h = (blockIdx.x / tiles) % a.Hq;
+  const int b = blockIdx.x / (tiles * a.Hq);
+  const int kvh = h / a.G;
+  Unit x;
+  decode_tile(a, nullptr, nullptr, b * tiles + qt, x);
+
+  if (tid == 0) {
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i == kBarP ? kBwdThreads : 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (tid < 32) {
+    tmem_alloc(smem_u32(tmem_ptr), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  const uint32_t lane_off = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+  const size_t row_base = static_cast<size_t>(b) * a.L;
+  const int t = x.m0 + tid;                           // this thread's query row
+
+  bool ok = true;
+  bool loads_out = false;
+  if (tid == 0) {
+    mbar_expect_tx(bar(kBarA), 2 * C::TILE);
+    load_tile<D>(sQ, &tq, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
+    load_tile<D>(sdO, &tdo, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
+  }
+  float dt = 0.f, l2 = 0.f;
+  if (t < a.L) {
+    const size_t off = ((row_base + t) * a.Hq + h) * D;
+    dt = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + off, static_cast<const __nv_bfloat16*>(ba.out) + off);
+    l2 = ba.lse[(static_cast<size_t>(b) * a.Hq + h) * a.L + t] * 1.4426950408889634f;
+  }
+  int j = 0;
+  for (; ok && j < x.n_tiles; ++j) {
+    const int n0 = tile_n0(x, j);
+    if (tid == 0) {
+      mbar_expect_tx(bar(kBarB), 2 * C::TILE);
+      load_tile<D>(sK, &tk, bar(kBarB), kvh, static_cast<int>(row_base) + n0);
+      load_tile<D>(sV, &tv, bar(kBarB), kvh, static_cast<int>(row_base) + n0);
+      loads_out = true;
+      ok = (j > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB), j & 1, a);
+      if (ok) {
+        loads_out = false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<false>(tmem, kmajor_desc<4>(sQ, kBM, kk), kmajor_desc<4>(sK, kBN, kk), C::IDESC_SS,
+                         kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<false>(tmem + 128, kmajor_desc<4>(sdO, kBM, kk), kmajor_desc<4>(sV, kBN, kk), C::IDESC_SS,
+                         kk > 0 ? 1u : 0u);
+        tc_commit(bar(kBarS));
+      }
+    }
+    __syncwarp();
+    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), j & 1, a)))) break;
+    tc_fence_after();
+    // dS of this query row, 64 key columns at a time, written over S
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      uint32_t sr[64], dr[64];
+      tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
+      tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
+      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
+      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
+      uint32_t dw[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = n0 + 64 * half + c + e;
+          const float p = visible(key, t, a) ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - l2) : 0.f;
+          ds[e] = p * (__uint_as_float(dr[c + e]) - dt);
+        }
+        dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st32(tmem + lane_off + 32 * half, dw);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar(kBarP));
+    if (tid == 0) {
+      if ((ok = bwd_wait(bar(kBarP), j & 1, a))) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::PV_STEPS; ++kk)
+          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(sK, kk), C::IDESC_ACC,
+                         (j == 0 && kk == 0) ? 0u : 1u);
+        tc_commit(bar(kBarO));
+      }
+    }
+    __syncwarp();
+    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), j & 1, a)))) break;
+  }
+  if (!ok && tid == 0) {
+    tc_commit(bar(kBarDrain));
+    bwd_wait(bar(kBarDrain), 0, a);
+    if (j == 0) bwd_wait(bar(kBarA), 0, a);
+    if (loads_out) bwd_wait(bar(kBarB), j & 1, a);
+  }
+  __syncwarp();
+  tc_fence_after();
+  if (__all_sync(0xffffffffu, ok)) {        // warp-uniform: the TMEM loads are warp-collective
+    const bool row_ok = t < a.L;
+    float* dq = ba.dq + ((row_base + (row_ok ? t : 0)) * a.Hq + h) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, r);
+      if (!row_ok) continue;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(dq + 32 * c + i) =
+            make_float4(__uint_as_float(r[i]) * a.scale, __uint_as_float(r[i + 1]) * a.scale,
+                        __uint_as_float(r[i + 2]) * a.scale, __uint_as_float(r[i + 3]) * a.scale);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid < 32) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  const PrefillArgs& a = ba.pa;
+  const long long tiles = (a.L + kBM - 1) / kBM;
+  const long long g_kv = tiles * a.Hkv * a.n_seq, g_q = tiles * a.Hq * a.n_seq;
+  if (g_kv == 0) return cudaSuccess;
+  if (g_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(swa_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(swa_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM (see SMEM_BYTES): refuse to launch if the occupancy says otherwise
+  static int checked = 0;
+  if (!checked) {
+    int n1 = 0, n2 = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, swa_bwd_dkdv_kernel<D>, kBwdThreads, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kBwdThreads, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (n1 != 1 || n2 != 1) return cudaErrorNotSupported;
+    checked = 1;
+  }
+  swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const BwdArgs& ba, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, int d, cudaStream_t stream) {
+  if (d == 64) return launch_bwd_impl<64>(ba, tq, tk, tv, tdo, stream);
+  if (d == 128) return launch_bwd_impl<128>(ba, tq, tk, tv, tdo, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace swa

@@ -36,6 +36,20 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
 
 // Two-query-tile prefill (heads 2p, 2p+1 per CTA); used when Hq is even and the
 // ring can hold two key tiles (always for 16 KB tiles, else when pairs share a KV head).
+// Backward pass: dq [n_seq, L, Hq, d], dk/dv [n_seq, L, Hkv, d] (fp32, written, not
+// accumulated) from q, k, v, the forward's out and lse and dout (bf16).
+struct BwdArgs {
+  PrefillArgs pa;       // geometry: n_seq sequences of length L, heads, window, sinks, scale
+  const void* out;      // [n_seq, L, Hq, d] bf16
+  const void* dout;     // [n_seq, L, Hq, d] bf16
+  const float* lse;     // [n_seq, Hq, L]
+  float* dq;
+  float* dk;
+  float* dv;
+};
+cudaError_t launch_bwd(const BwdArgs& ba, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, int d, cudaStream_t stream);
+
 // Short-window stream kernel: d = 64, bf16 inputs, window <= 129, no sink prefix.
 bool prefill_stream_supported(int d, bool f32, int window, int n_sink);
 cudaError_t launch_prefill_stream(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,

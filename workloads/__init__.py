@@ -255,6 +255,12 @@ class ProjWorkload:
                 "in_dtype": "bf16", "out_dtype": self.out_dtype}
 
 
+# backward passes: (forward workload, sequence length or None for the workload's own)
+BWD_WORKLOADS = {
+    "bwd_based_local": ("based_local", None),
+    "bwd_gqa8b_L8192": ("gqa8b_prefill", 8192),
+}
+
 ROPE_WORKLOADS = {
     # rotary encoding of the 8B-shaped prefill's q and k before attention
     "rope_qk_gqa8b": dict(T=32768, Hq=32, Hkv=8, d=128, rope_base=10000.0),
