@@ -203,12 +203,13 @@ def load_peaks():
         return dict(PEAKS_FALLBACK, source="fallback")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files=None) -> str:
+    """Hash of the kernel sources (all of them, or the named files of csrc/)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sink_aware_sliding_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    names = sorted(files) if files else sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h")))
+    for name in names:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -221,7 +222,7 @@ def profiled_traffic(workload: str):
     except Exception:
         return None
     e = d.get(workload)
-    if not e or e.get("kernel_hash") != kernel_source_hash():
+    if not e or e.get("kernel_hash") != kernel_source_hash(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -714,6 +715,23 @@ def profile_case(args):
         for _ in range(n):
             swa.swa_hadamard_proj(y, alpha, beta, z)
         torch.cuda.synchronize()
+        return
+    if args.profile_case in wl.BWD_WORKLOADS:
+        fwd_name, L = wl.BWD_WORKLOADS[args.profile_case]
+        w = wl.WORKLOADS[fwd_name]
+        q, k, v = wl.make_prefill(w, device=dev, L=args.L or L)
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[0], w.Hq, q.shape[1], device=dev, dtype=torch.float32)
+        swa.swa_fwd(q, k, v, out, lse, w.window, w.n_sink)
+        do = torch.randn_like(q)
+        dq = torch.empty(q.shape, device=dev)
+        dk = torch.empty(k.shape, device=dev)
+        dv = torch.empty_like(dk)
+        for _ in range(n):
+            swa.swa_bwd(q, k, v, out, do, lse, dq, dk, dv, w.window, w.n_sink)
+        torch.cuda.synchronize()
+        if swa.swa_device_error() != 0:
+            raise SystemExit("device wait timed out")
         return
     if args.profile_case in wl.ROPE_WORKLOADS:
         c = wl.ROPE_WORKLOADS[args.profile_case]
