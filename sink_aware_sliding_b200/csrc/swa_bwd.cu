@@ -15,13 +15,18 @@
 //   swa_bwd_dq_kernel    one CTA per (sequence, query head, 128-row query tile): for
 //                        the key tiles the forward visits it computes S and dP, forms
 //                        dS per query row and accumulates dQ += dS K in TMEM.
+// A third, small kernel computes D_t = rowsum(dO_t O_t) for every row first,
+// into the storage of dq (which the dQ kernel only writes after the dK/dV kernel
+// has read D; the dQ kernel forms its own D per row).
 // Each CTA is one warpgroup; thread 0 issues TMA and MMA, all threads do the
 // element-wise step; every hand-off is an mbarrier with a bounded wait.  Thread 0
 // shares warp 0 with element-wise threads, so the warp is reconverged
 // (__syncwarp) after every issuer-only block and every wait's outcome is made
-// warp-uniform before the warp-collective tcgen05 instructions that follow.  This is
-// the first, non-overlapped version: loads, products and the element-wise step of
-// one tile pair run one after another.
+// warp-uniform before the warp-collective tcgen05 instructions that follow.  The
+// tiles that change per iteration (Q and dO, or K and V) are double-buffered and
+// the next iteration's are requested when the current one starts; the products
+// and the element-wise step of one iteration still run one after another (TMEM
+// holds one iteration's S^T and dP^T next to the accumulators).
 //
 // TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
 // written over their first halves), dV 256.., dK 256+d..; (dQ kernel): S 0-127,
@@ -30,6 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "prefill_common.cuh"
@@ -47,9 +53,10 @@ struct BwdCfg {
   static constexpr int NCHUNK = D / 64;                // 128-byte column chunks
   static constexpr int QK_STEPS = D / 16;
   static constexpr int PV_STEPS = kBN / 16;
-  // shared layout: tiles 0..3, then D_s, L_s (128 floats each), then barriers
+  // shared layout: tiles 0..5 (two fixed, two double-buffered), then D_s, L_s
+  // (128 floats each), then barriers
   static constexpr int OFF_T = 0;
-  static constexpr int OFF_DS = 4 * TILE;
+  static constexpr int OFF_DS = 6 * TILE;
   static constexpr int OFF_LS = OFF_DS + 512;
   static constexpr int OFF_BAR = OFF_LS + 512;
   static constexpr int NBAR = 8;
@@ -65,12 +72,12 @@ struct BwdCfg {
 
 // barrier indices
 constexpr int kBarA = 0;      // K,V (dK/dV kernel) or Q,dO (dQ kernel): loaded once
-constexpr int kBarB = 1;      // the per-iteration tile pair
-constexpr int kBarS = 2;      // both score products done
-constexpr int kBarP = 3;      // all 128 rows wrote their P / dS (count 128)
-constexpr int kBarO = 4;      // accumulation products done
-constexpr int kBarRow = 5;    // per-iteration row data (D, lse) written (count 128)
-constexpr int kBarDrain = 6;
+constexpr int kBarB = 1;      // the per-iteration tile pair, buffers 0 and 1 (kBarB, kBarB + 1)
+constexpr int kBarS = 3;      // both score products done
+constexpr int kBarP = 4;      // all 128 rows wrote their P / dS (count 128)
+constexpr int kBarO = 5;      // accumulation products done
+constexpr int kBarRow = 6;    // per-iteration row data (D, lse) written (count 128)
+constexpr int kBarDrain = 7;
 
 __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const PrefillArgs& a) {
   for (int i = 0; i < 256; ++i)
@@ -111,6 +118,22 @@ template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int head, int row) {
 #pragma unroll
   for (int c = 0; c < BwdCfg<D>::NCHUNK; ++c) tma_load_3d(dst + c * (kBM * 128), map, bar, c * 64, head, row);
+}
+
+// ------------------------------------------------------------------ D
+// D[(b * Hq + h) * L + t] = rowsum(dout * out) of row (b, t, h), one thread per row.
+template <int D>
+__global__ void __launch_bounds__(256) swa_bwd_dot_kernel(const __grid_constant__ BwdArgs ba) {
+  const PrefillArgs& a = ba.pa;
+  const long long rows = static_cast<long long>(a.n_seq) * a.L * a.Hq;
+  for (long long r = blockIdx.x * 256LL + threadIdx.x; r < rows; r += static_cast<long long>(gridDim.x) * 256) {
+    const int h = static_cast<int>(r % a.Hq);
+    const long long bt = r / a.Hq;
+    const int t = static_cast<int>(bt % a.L);
+    const long long b = bt / a.L;
+    ba.dq[(b * a.Hq + h) * a.L + t] = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + r * D,
+                                                  static_cast<const __nv_bfloat16*>(ba.out) + r * D);
+  }
 }
 
 // ------------------------------------------------------------------ dK, dV
@@ -156,111 +179,128 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t lane_off = static_cast<uint32_t>((tid >> 5) * 32) << 16;
   const size_t row_base = static_cast<size_t>(b) * a.L;
 
+  // iterations: (query head g, query tile) flattened, query tiles fastest
+  const int nq = it_hi - jt + 1;
+  const int n_it = a.G * nq;
+  auto it_head = [&](int i) { return kvh * a.G + i / nq; };
+  auto it_row0 = [&](int i) { return (jt + i % nq) * kBM; };
+  auto issue = [&](int i) {                           // thread 0: Q, dO of iteration i
+    const int buf = i & 1;
+    mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
+    load_tile<D>(sQ + 2 * buf * C::TILE, &tq, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
+    load_tile<D>(sdO + 2 * buf * C::TILE, &tdo, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
+  };
+  const float* d_rows = ba.dq;                        // D, written by the D kernel
+  auto fetch_row = [&](int i, float& dt, float& l2) { // D and lse (log2 units) of query it_row0(i) + tid
+    const int t = it_row0(i) + tid;
+    const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + t;
+    dt = t < a.L ? d_rows[idx] : 0.f;
+    l2 = t < a.L ? ba.lse[idx] * 1.4426950408889634f : 0.f;
+  };
+
   bool ok = true;
-  bool loads_out = false;
+  int issued = 0;                                     // iterations whose tiles were requested
   if (tid == 0) {
     mbar_expect_tx(bar(kBarA), 2 * C::TILE);
     load_tile<D>(sK, &tk, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
     load_tile<D>(sV, &tv, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
+    issue(0);
+    issued = 1;
   }
-  int it = 0;
+  float next_d = 0.f, next_l = 0.f;
+  fetch_row(0, next_d, next_l);
+  D_s[tid] = next_d;
+  L_s[tid] = next_l;
+  mbar_arrive(bar(kBarRow));
   const int s_key = j0 + tid;                         // this thread's key (TMEM lane)
-  for (int g = 0; ok && g < a.G; ++g) {
-    const int h = kvh * a.G + g;
-    for (int qi = jt; ok && qi <= it_hi; ++qi, ++it) {
-      const int i0 = qi * kBM;
-      if (tid == 0) {
-        mbar_expect_tx(bar(kBarB), 2 * C::TILE);
-        load_tile<D>(sQ, &tq, bar(kBarB), h, static_cast<int>(row_base) + i0);
-        load_tile<D>(sdO, &tdo, bar(kBarB), h, static_cast<int>(row_base) + i0);
-        loads_out = true;
-      }
-      {  // D and log-sum-exp (log2 units) of query i0 + tid
-        const int t = i0 + tid;
-        float dt = 0.f, l2 = 0.f;
-        if (t < a.L) {
-          const size_t off = ((row_base + t) * a.Hq + h) * D;
-          dt = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + off,
-                          static_cast<const __nv_bfloat16*>(ba.out) + off);
-          l2 = ba.lse[(static_cast<size_t>(b) * a.Hq + h) * a.L + t] * 1.4426950408889634f;
-        }
-        D_s[tid] = dt;
-        L_s[tid] = l2;
-        mbar_arrive(bar(kBarRow));
-      }
-      __syncwarp();
-      if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
-      if (tid == 0) {
-        ok = (it > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB), it & 1, a);
-        if (ok) {
-          loads_out = false;
-          tc_fence_after();
+  int it = 0;
+  for (; it < n_it; ++it) {
+    const int i0 = it_row0(it), buf = it & 1;
+    const uint32_t cQ = sQ + 2 * buf * C::TILE, cdO = sdO + 2 * buf * C::TILE;
+    // the next iteration's tiles (its buffer's last readers finished with the
+    // previous iteration) and row data (kept in registers until this one is done)
+    if (tid == 0 && it + 1 < n_it) {
+      issue(it + 1);
+      issued = it + 2;
+    }
+    if (it + 1 < n_it) fetch_row(it + 1, next_d, next_l);
+    __syncwarp();
+    if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
+    if (tid == 0) {
+      ok = (it > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB + buf), (it >> 1) & 1, a);
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < C::QK_STEPS; ++kk)
-            umma_ss<false>(tmem, kmajor_desc<4>(sK, kBN, kk), kmajor_desc<4>(sQ, kBM, kk), C::IDESC_SS,
-                           kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<false>(tmem, kmajor_desc<4>(sK, kBN, kk), kmajor_desc<4>(cQ, kBM, kk), C::IDESC_SS,
+                         kk > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < C::QK_STEPS; ++kk)
-            umma_ss<false>(tmem + 128, kmajor_desc<4>(sV, kBN, kk), kmajor_desc<4>(sdO, kBM, kk), C::IDESC_SS,
-                           kk > 0 ? 1u : 0u);
-          tc_commit(bar(kBarS));
-        }
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<false>(tmem + 128, kmajor_desc<4>(sV, kBN, kk), kmajor_desc<4>(cdO, kBM, kk), C::IDESC_SS,
+                         kk > 0 ? 1u : 0u);
+        tc_commit(bar(kBarS));
       }
-      __syncwarp();
-      if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), it & 1, a)))) break;
-      tc_fence_after();
-      // P^T and dS^T of this key row, 64 query columns at a time
+    }
+    __syncwarp();
+    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), it & 1, a)))) break;
+    tc_fence_after();
+    // P^T and dS^T of this key row, 64 query columns at a time
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64], dr[64];
-        tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
-        tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
-        tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
-        tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
-        uint32_t pw[32], dw[32];
+    for (int half = 0; half < 2; ++half) {
+      uint32_t sr[64], dr[64];
+      tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
+      tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
+      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
+      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
+      uint32_t pw[32], dw[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float p[2], ds[2];
+      for (int c = 0; c < 64; c += 2) {
+        float p[2], ds[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 64 * half + c + e;
-            const bool vis = visible(s_key, i0 + col, a);
-            p[e] = vis ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]) : 0.f;
-            ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
-          }
-          pw[c / 2] = pack_bf16x2(p[0], p[1]);
-          dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+        for (int e = 0; e < 2; ++e) {
+          const int col = 64 * half + c + e;
+          const bool vis = visible(s_key, i0 + col, a);
+          p[e] = vis ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]) : 0.f;
+          ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
         }
-        tmem_st32(tmem + lane_off + 32 * half, pw);
-        tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
+        pw[c / 2] = pack_bf16x2(p[0], p[1]);
+        dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarP));
-      if (tid == 0) {
-        if ((ok = bwd_wait(bar(kBarP), it & 1, a))) {
-          tc_fence_after();
+      tmem_st32(tmem + lane_off + 32 * half, pw);
+      tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar(kBarP));
+    if (tid == 0) {
+      if ((ok = bwd_wait(bar(kBarP), it & 1, a))) {
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < C::PV_STEPS; ++kk)
-            umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(sdO, kk), C::IDESC_ACC,
-                           (it == 0 && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < C::PV_STEPS; ++kk)
+          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(cdO, kk), C::IDESC_ACC,
+                         (it == 0 && kk == 0) ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < C::PV_STEPS; ++kk)
-            umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, v_desc<false, 16>(sQ, kk), C::IDESC_ACC,
-                           (it == 0 && kk == 0) ? 0u : 1u);
-          tc_commit(bar(kBarO));
-        }
+        for (int kk = 0; kk < C::PV_STEPS; ++kk)
+          umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, v_desc<false, 16>(cQ, kk), C::IDESC_ACC,
+                         (it == 0 && kk == 0) ? 0u : 1u);
+        tc_commit(bar(kBarO));
       }
-      __syncwarp();
-      if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
+    }
+    __syncwarp();
+    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
+    // every thread is past this iteration's element-wise step: publish the next row data
+    if (it + 1 < n_it) {
+      D_s[tid] = next_d;
+      L_s[tid] = next_l;
+      mbar_arrive(bar(kBarRow));
     }
   }
   if (!ok && tid == 0) {
     // let everything this thread started finish before the CTA releases its memory
     tc_commit(bar(kBarDrain));
     bwd_wait(bar(kBarDrain), 0, a);
-    if (it == 0) bwd_wait(bar(kBarA), 0, a);
-    if (loads_out) bwd_wait(bar(kBarB), it & 1, a);
+    bwd_wait(bar(kBarA), 0, a);
+    for (int i = it; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
   }
   __syncwarp();
   tc_fence_after();
@@ -333,11 +373,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int t = x.m0 + tid;                           // this thread's query row
 
   bool ok = true;
-  bool loads_out = false;
+  int issued = 0;                                     // key tiles whose K, V were requested
+  auto issue = [&](int jj) {                          // thread 0: K, V of key tile step jj
+    const int buf = jj & 1, n0 = tile_n0(x, jj);
+    mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
+    load_tile<D>(sK + 2 * buf * C::TILE, &tk, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
+    load_tile<D>(sV + 2 * buf * C::TILE, &tv, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
+  };
   if (tid == 0) {
     mbar_expect_tx(bar(kBarA), 2 * C::TILE);
     load_tile<D>(sQ, &tq, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
     load_tile<D>(sdO, &tdo, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
+    issue(0);
+    issued = 1;
   }
   float dt = 0.f, l2 = 0.f;
   if (t < a.L) {
@@ -347,23 +395,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   int j = 0;
   for (; ok && j < x.n_tiles; ++j) {
-    const int n0 = tile_n0(x, j);
+    const int n0 = tile_n0(x, j), buf = j & 1;
+    const uint32_t cK = sK + 2 * buf * C::TILE, cV = sV + 2 * buf * C::TILE;
     if (tid == 0) {
-      mbar_expect_tx(bar(kBarB), 2 * C::TILE);
-      load_tile<D>(sK, &tk, bar(kBarB), kvh, static_cast<int>(row_base) + n0);
-      load_tile<D>(sV, &tv, bar(kBarB), kvh, static_cast<int>(row_base) + n0);
-      loads_out = true;
-      ok = (j > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB), j & 1, a);
+      // the next key tile's K, V: its buffer's last readers finished with step j-1
+      if (j + 1 < x.n_tiles) {
+        issue(j + 1);
+        issued = j + 2;
+      }
+      ok = (j > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB + buf), (j >> 1) & 1, a);
       if (ok) {
-        loads_out = false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem, kmajor_desc<4>(sQ, kBM, kk), kmajor_desc<4>(sK, kBN, kk), C::IDESC_SS,
+          umma_ss<false>(tmem, kmajor_desc<4>(sQ, kBM, kk), kmajor_desc<4>(cK, kBN, kk), C::IDESC_SS,
                          kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem + 128, kmajor_desc<4>(sdO, kBM, kk), kmajor_desc<4>(sV, kBN, kk), C::IDESC_SS,
+          umma_ss<false>(tmem + 128, kmajor_desc<4>(sdO, kBM, kk), kmajor_desc<4>(cV, kBN, kk), C::IDESC_SS,
                          kk > 0 ? 1u : 0u);
         tc_commit(bar(kBarS));
       }
@@ -401,7 +450,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(sK, kk), C::IDESC_ACC,
+          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(cK, kk), C::IDESC_ACC,
                          (j == 0 && kk == 0) ? 0u : 1u);
         tc_commit(bar(kBarO));
       }
@@ -412,8 +461,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (!ok && tid == 0) {
     tc_commit(bar(kBarDrain));
     bwd_wait(bar(kBarDrain), 0, a);
-    if (j == 0) bwd_wait(bar(kBarA), 0, a);
-    if (loads_out) bwd_wait(bar(kBarB), j & 1, a);
+    bwd_wait(bar(kBarA), 0, a);
+    for (int i = j; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
   }
   __syncwarp();
   tc_fence_after();
@@ -463,6 +512,10 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
     if (n1 != 1 || n2 != 1) return cudaErrorNotSupported;
     checked = 1;
   }
+  const long long rows = static_cast<long long>(a.n_seq) * a.L * a.Hq;
+  swa_bwd_dot_kernel<D><<<static_cast<unsigned>(std::min<long long>((rows + 255) / 256, 148LL * 32)), 256, 0, stream>>>(ba);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
