@@ -12,6 +12,15 @@
 // alternate query tiles and run independently, so one tile's softmax and
 // epilogue overlap the other's.
 //
+// The products run on 64-key sub-tiles (halves of the 128-key tiles in shared
+// memory, addressed by descriptor offsets).  Each warpgroup's 128-column S region
+// holds two sub-tiles' S: the P of sub-tile g (packed bf16) occupies the first 32
+// columns of its half, so S of sub-tile g+1 is computed into the other half while
+// the warpgroup works on g, and the softmax finds its next S ready instead of
+// waiting for P V -> Q K^T to round-trip.  A warp none of whose rows sees any key
+// of a sub-tile skips it (with a 128-key window every warp skips one of the four
+// sub-tiles of a query tile).
+//
 // Roles (384 threads):
 //   warps 0-3   softmax + epilogue of the even query tiles of the range (A)
 //   warps 4-7   the odd ones (B)
@@ -20,18 +29,19 @@
 //   warps 9, 10 tcgen05.mma issue, one thread for each softmax warpgroup (warp 9
 //               also allocates TMEM): a tcgen05.mma issue stalls while the tensor
 //               pipe is backed up, so one issuer per warpgroup keeps either from
-//               waiting on the other's issue.  A commit covers the issuing
-//               thread's own MMAs, which execute in issue order, so "S ready"
-//               still implies that warpgroup's previous P V has finished.
+//               waiting on the other's issue.  Per sub-tile g it issues S(g+1)
+//               (into the half P(g-1) has left), waits for P(g), then O += P(g) V.
 // A key-tile slot is freed after two arrivals: one commit per query tile that
 // used it, plus an immediate arrive when only one query tile of the range uses
 // it (the first tile of a range, or the last tile of a sequence).
+// Barriers per warpgroup: S ready and P written, one per S half (so no wait can
+// confuse two completed phases); a P V done barrier that the softmax waits on
+// only to rescale O (S(g) ready implies P V of g-2 has finished, so that wait is
+// unambiguous too); O final, one per O buffer.
 // TMEM columns: S_A 0-127, S_B 128-255, then two O buffers per warpgroup (64
 // columns each: O_A 256/320, O_B 384/448).  Query tile k of a warpgroup
 // accumulates into buffer k mod 2, so the warpgroup writes out tile k-1 (its
-// epilogue) while the tensor pipe computes tile k's second S: the epilogue fills
-// the wait for S instead of adding to it.  Each O buffer has its own "final"
-// barrier, so a wait can never confuse two completed phases.
+// epilogue) while the tensor pipe computes tile k.
 // With bf16 output, a finished query tile's Q slot is its output staging tile
 // (TMA store), as in the pair kernel.
 #include <cuda.h>
@@ -65,18 +75,19 @@ struct StreamCfg {
   static constexpr int NKV = 4;                     // key-tile ring (K and V per slot)
   static constexpr int KSTEP = 16;                  // K of one bf16 MMA (32 bytes)
   static constexpr int QK_STEPS = D / KSTEP;
-  static constexpr int PV_STEPS = kBN / KSTEP;
+  static constexpr int SUB = 64;                    // keys per sub-tile (half a key tile)
+  static constexpr int PV_STEPS = SUB / KSTEP;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + NQ * TILE;
   static constexpr int OFF_BAR = OFF_KV + NKV * 2 * TILE;
   static constexpr int B_QFULL = 0, B_QEMPTY = NQ, B_KVFULL = 2 * NQ, B_KVEMPTY = 2 * NQ + NKV,
-                       B_SFULL = 2 * NQ + 2 * NKV, B_PFULL = B_SFULL + 2, B_OFINAL = B_PFULL + 2,
-                       B_DRAIN = B_OFINAL + 4, NBAR = B_DRAIN + 2;
+                       B_SFULL = 2 * NQ + 2 * NKV, B_PFULL = B_SFULL + 4, B_PVDONE = B_PFULL + 4,
+                       B_OFINAL = B_PVDONE + 2, B_DRAIN = B_OFINAL + 4, NBAR = B_DRAIN + 2;
   static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEMPTR + 4;
   static constexpr int OFF_TABLES = OFF_ABORT + 12;
   static constexpr int SMEM_BYTES = OFF_TABLES + 2 * 4 * (kMaxSeqSmem + 1) + 1024;
-  static constexpr uint32_t IDESC_QK = make_idesc(1u, kBM, kBN, false);
+  static constexpr uint32_t IDESC_QK = make_idesc(1u, kBM, SUB, false);
   static constexpr uint32_t IDESC_PV = make_idesc(1u, kBM, D, true);
   __device__ static constexpr uint32_t tmem_s(int x) { return x ? 128u : 0u; }
   __device__ static constexpr uint32_t tmem_o(int x, int ob) { return 256u + 2 * D * x + D * ob; }
@@ -113,11 +124,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       mbar_init(bar(C::B_KVFULL + i), 1);
       mbar_init(bar(C::B_KVEMPTY + i), 2);    // two users, or one user and a stand-in arrive
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {          // per warpgroup and S half / O buffer
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 128);
-      mbar_init(bar(C::B_OFINAL + 2 * i), 1);
-      mbar_init(bar(C::B_OFINAL + 2 * i + 1), 1);
+      mbar_init(bar(C::B_OFINAL + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_PVDONE + i), 1);
       mbar_init(bar(C::B_DRAIN + i), 1);
     }
     *abort_flag = 0;
@@ -212,57 +225,85 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int x = warp - kStreamMmaWarp;             // the softmax warpgroup this thread serves
     if (lane == 0 && x < n_range) {
       bool ok = true;
-      int pcnt = 0;
       const uint32_t s_t = tmem + C::tmem_s(x);
-      // per-tile plan; the next tile's is worked out while this thread waits for
-      // the warpgroup's last P of the current one
-      struct Plan {
-        int nt, last_kc;
+      // this warpgroup's 64-key sub-tiles in order: query tiles li = x, x+2, ...,
+      // within each the sub-tiles f64 .. l64 of its band
+      struct Sub {
+        int li, k;                   // range tile, its index among this warpgroup's tiles
+        int s64, f64, l64;           // current, first and last sub-tile of the tile
+        int m, last_kc;              // diagonal key tile and its ring counter
         bool single_prev, single_diag;
       };
-      auto plan_of = [&](int li) {
-        Plan pl;
-        Unit u;
+      auto start_tile = [&](Sub& u, int li, int k) -> bool {
+        u.li = li;
+        u.k = k;
+        if (li >= n_range) return false;
+        Unit t;
         int h, seq_tiles;
-        qtile(li, u, h, seq_tiles);
-        const int qt = u.m0 / kBM;
-        pl.nt = u.n_tiles;
-        pl.last_kc = li + extra;
-        pl.single_prev = !(li > 0 && qt > 0);
-        pl.single_diag = !(li + 1 < n_range && qt + 1 < seq_tiles && a.window > 1);
-        return pl;
+        qtile(li, t, h, seq_tiles);
+        const int qt = t.m0 / kBM;
+        u.f64 = max(0, t.m0 - a.window + 1) / C::SUB;
+        u.l64 = t.m1 / C::SUB;
+        u.s64 = u.f64;
+        u.m = t.m1 / kBN;
+        u.last_kc = li + extra;
+        u.single_prev = !(li > 0 && qt > 0);
+        u.single_diag = !(li + 1 < n_range && qt + 1 < seq_tiles && a.window > 1);
+        return true;
       };
-      Plan cur = plan_of(x);
-      for (int li = x, k = 0; ok && li < n_range; li += 2, ++k) {
-        Plan nxt = cur;
-        const uint32_t o_t = tmem + C::tmem_o(x, k & 1);
-        const uint32_t q_tile = base + C::OFF_Q + (li % C::NQ) * C::TILE;
-        if (!(ok = wait_bar(bar(C::B_QFULL + li % C::NQ), (li / C::NQ) & 1, ctl))) break;
-        for (int j = 0; j < cur.nt; ++j) {
-          const int kc = cur.last_kc - (cur.nt - 1 - j);
-          const uint32_t kv = base + C::OFF_KV + (kc % C::NKV) * 2 * C::TILE;
-          // S = Q K^T (the S region is free: this thread's previous P V was issued before)
-          if (!(ok = wait_bar(bar(C::B_KVFULL + kc % C::NKV), (kc / C::NKV) & 1, ctl))) break;
-          tc_fence_after();
+      auto advance = [&](const Sub& u, Sub& v) -> bool {
+        v = u;
+        if (u.s64 < u.l64) {
+          v.s64 = u.s64 + 1;
+          return true;
+        }
+        return start_tile(v, u.li + 2, u.k + 1);
+      };
+      auto kc_of = [&](const Sub& u) { return u.last_kc - (u.m - (u.s64 >> 1)); };
+      // S of sub-tile u = Q K_u^T into half `half` of this warpgroup's S region
+      auto issue_qk = [&](const Sub& u, int half) -> bool {
+        const int kc = kc_of(u);
+        if (u.s64 == u.f64 && !wait_bar(bar(C::B_QFULL + u.li % C::NQ), (u.li / C::NQ) & 1, ctl)) return false;
+        if (!wait_bar(bar(C::B_KVFULL + kc % C::NKV), (kc / C::NKV) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t q_tile = base + C::OFF_Q + (u.li % C::NQ) * C::TILE;
+        const uint32_t k_sub = base + C::OFF_KV + (kc % C::NKV) * 2 * C::TILE + (u.s64 & 1) * (C::SUB * 128);
 #pragma unroll
-          for (int kk = 0; kk < C::QK_STEPS; ++kk)
-            umma_ss<false>(s_t, kmajor_desc<C::QK_STEPS>(q_tile, kBM, kk), kmajor_desc<C::QK_STEPS>(kv, kBN, kk),
-                           C::IDESC_QK, kk > 0 ? 1u : 0u);
-          tc_commit(bar(C::B_SFULL + x));
-          if (j == cur.nt - 1 && li + 2 < n_range) nxt = plan_of(li + 2);
-          // O += P V once the warpgroup has written P over S
-          if (!(ok = wait_bar(bar(C::B_PFULL + x), pcnt & 1, ctl))) break;
-          ++pcnt;
+        for (int kk = 0; kk < C::QK_STEPS; ++kk)
+          umma_ss<false>(s_t + C::SUB * half, kmajor_desc<C::QK_STEPS>(q_tile, kBM, kk),
+                         kmajor_desc<C::QK_STEPS>(k_sub, C::SUB, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+        tc_commit(bar(C::B_SFULL + 2 * x + half));
+        return true;
+      };
+      Sub cur;
+      if (start_tile(cur, x, 0)) {
+        ok = issue_qk(cur, 0);
+        for (int g = 0; ok; ++g) {
+          // one sub-tile ahead: the next S goes into the other half, whose P the
+          // previous P V (issued last round, executed in order) has consumed
+          Sub nxt;
+          const bool more = advance(cur, nxt);
+          if (more && !(ok = issue_qk(nxt, (g + 1) & 1))) break;
+          if (!(ok = wait_bar(bar(C::B_PFULL + 2 * x + (g & 1)), (g >> 1) & 1, ctl))) break;
           tc_fence_after();
+          const int kc = kc_of(cur);
+          const uint32_t v_tile = base + C::OFF_KV + (kc % C::NKV) * 2 * C::TILE + C::TILE;
+          const uint32_t o_t = tmem + C::tmem_o(x, cur.k & 1);
 #pragma unroll
           for (int kk = 0; kk < C::PV_STEPS; ++kk)
-            umma_ts<false>(o_t, s_t + kk * 8, v_desc<false, C::KSTEP>(kv + C::TILE, kk), C::IDESC_PV,
-                           (j == 0 && kk == 0) ? 0u : 1u);
-          tc_commit(bar(C::B_KVEMPTY + kc % C::NKV));
-          if (j == cur.nt - 1 ? cur.single_diag : cur.single_prev) mbar_arrive(bar(C::B_KVEMPTY + kc % C::NKV));
+            umma_ts<false>(o_t, s_t + C::SUB * (g & 1) + kk * 8,
+                           v_desc<false, C::KSTEP>(v_tile, kk + C::PV_STEPS * (cur.s64 & 1)), C::IDESC_PV,
+                           (cur.s64 == cur.f64 && kk == 0) ? 0u : 1u);
+          tc_commit(bar(C::B_PVDONE + x));
+          if ((cur.s64 & 1) || cur.s64 == cur.l64) {     // this tile's last use of the key tile
+            tc_commit(bar(C::B_KVEMPTY + kc % C::NKV));
+            if ((cur.s64 >> 1) == cur.m ? cur.single_diag : cur.single_prev)
+              mbar_arrive(bar(C::B_KVEMPTY + kc % C::NKV));
+          }
+          if (cur.s64 == cur.l64) tc_commit(bar(C::B_OFINAL + 2 * x + (cur.k & 1)));
+          if (!more) break;
+          cur = nxt;
         }
-        if (ok) tc_commit(bar(C::B_OFINAL + 2 * x + (k & 1)));
-        cur = nxt;
       }
       if (*abort_flag) {
         // Every MMA this thread issued must finish before TMEM is freed.
@@ -279,7 +320,6 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int r = tid & 127;                         // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tmem = tmem + C::tmem_s(x_wg) + lane_off;
-    int scnt = 0;
     bool ok = true;
     // the previous query tile of this warpgroup, written out one step late
     bool have_prev = false;
@@ -311,25 +351,36 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       }
       return true;
     };
+    int g = 0;                                       // this warpgroup's sub-tiles so far
     for (int li = x_wg, k = 0; ok && li < n_range; li += 2, ++k) {
       Unit x;
       int h, seq_tiles;
       qtile(li, x, h, seq_tiles);
       const int t = x.m0 + r;
       const uint32_t o_tmem = tmem + C::tmem_o(x_wg, k & 1) + lane_off;
+      const int f64 = max(0, x.m0 - a.window + 1) / C::SUB, l64 = x.m1 / C::SUB;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < x.n_tiles; ++j, ++scnt) {
-        ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SFULL + x_wg), scnt & 1, ctl));
+      for (int s64 = f64; s64 <= l64; ++s64, ++g) {
+        const int half = g & 1;
+        ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SFULL + 2 * x_wg + half), (g >> 1) & 1, ctl));
         if (!ok) break;
         tc_fence_after();
         float alpha;
-        const bool need = softmax_tile<false>(s_tmem, x, j, t, a, m_run, l_run, alpha);
-        // O += P(j-1) V(j-1) has finished (it was issued before S(j)).
-        if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<D>(o_tmem, alpha);
+        const int n0 = s64 * C::SUB;
+        const bool need = softmax_sub64(s_tmem + C::SUB * half, t - a.window + 1 - n0, t - n0, a.scale_log2,
+                                        m_run, l_run, alpha);
+        if (s64 > f64 && __any_sync(0xffffffffu, need)) {
+          // O holds the products of the earlier sub-tiles: wait for the last one
+          // (S of this sub-tile being ready implies the one before it has finished)
+          ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_PVDONE + x_wg), (g - 1) & 1, ctl));
+          if (!ok) break;
+          tc_fence_after();
+          rescale_o<D>(o_tmem, alpha);
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(C::B_PFULL + x_wg));
-        if (j == 0 && have_prev) {
+        mbar_arrive(bar(C::B_PFULL + 2 * x_wg + half));
+        if (s64 == f64 && have_prev) {
           // the previous tile's epilogue, while the tensor pipe works on this one
           if (!(ok = epilogue())) break;
           have_prev = false;

@@ -3,9 +3,9 @@
 
 Every case is checked against the oracle, and, where the pair kernel applies (an
 even head count), against it on the same inputs (debug flag 4 turns the stream
-kernel off): the two kernels run the
-same tcgen05 products and the same per-tile softmax in the same key order, so
-their outputs must agree bit for bit.  The ranges of query tiles a CTA streams
+kernel off).  The stream kernel works on 64-key sub-tiles and the pair kernel on
+128-key tiles, so their running maxima and summation orders differ and the two
+agree within the oracle bounds, not bit for bit.  The ranges of query tiles a CTA streams
 cross heads and sequences, start in the middle of sequences and can be a single
 tile; the cases below make all of that happen."""
 import math
@@ -78,8 +78,8 @@ def test_stream_matches_oracle_and_pair_kernel(B, L, Hq, Hkv, window):
         assert_close(lse, rl, f"stream lse[{od}]")
         if Hq % 2 == 0:                     # the pair kernel applies (odd Hq: one-tile kernel)
             pout, plse = run(qd, kd, vd, window, od, flag=4)
-            assert torch.equal(out, pout), "stream and pair kernels differ (out)"
-            assert torch.equal(lse, plse), "stream and pair kernels differ (lse)"
+            assert_close(out, pout.double().cpu(), f"stream vs pair out[{od}]", max_abs=max_abs)
+            assert_close(lse, plse.double().cpu(), f"stream vs pair lse[{od}]")
 
 
 def test_stream_varlen_matches_oracle():
@@ -104,16 +104,17 @@ def test_stream_varlen_matches_oracle():
             assert_close(lse, rl, f"varlen lse[{od}, flag {flag}]")
 
 
-def test_based_local_stream_equals_pair_kernel():
-    """The benchmark workload in its launch configuration: the stream kernel's output
-    equals the pair kernel's bit for bit (the pair kernel is checked against the
-    oracle at this size in the prefill tests)."""
+def test_based_local_stream_against_pair_kernel():
+    """The benchmark workload in its launch configuration: every element of the
+    stream kernel's output against the pair kernel's (checked against the oracle at
+    this size in the prefill tests), and sampled rows against the oracle."""
     w = WORKLOADS["based_local"]
     q, k, v = workloads.make_prefill(w, device="cuda")
-    out, lse = run(q, k, v, w.window, torch.bfloat16)
-    pout, plse = run(q, k, v, w.window, torch.bfloat16, flag=4)
-    assert torch.equal(out, pout)
-    assert torch.equal(lse, plse)
+    out, lse = run(q, k, v, w.window, torch.float32)
+    pout, plse = run(q, k, v, w.window, torch.float32, flag=4)
+    err = (out - pout).abs()
+    assert err.max().item() <= 1e-2 and err.mean().item() <= 1e-3
+    assert (lse - plse).abs().max().item() <= 1e-2
     rows = workloads.sample_rows(w.L, w.window, w.n_sink, n_random=64)
     for b in (0, w.B - 1):
         ro, rl = oracle.swa_rows(q[b, rows].cpu(), rows, k[b].cpu(), v[b].cpu(), w.window, 0, w.scale)
