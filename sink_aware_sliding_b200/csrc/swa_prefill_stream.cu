@@ -93,6 +93,68 @@ struct StreamCfg {
   __device__ static constexpr uint32_t tmem_o(int x, int ob) { return 256u + 2 * D * x + D * ob; }
 };
 
+// The online-softmax step of softmax_tile on a 64-key sub-tile (no sink prefix in
+// it): visible columns lo .. hi relative to the sub-tile's first key.  P is
+// written over the first 32 columns of the sub-tile's S (packed bf16 pairs).
+// A warp none of whose rows sees any key of the sub-tile only writes zeros.  The
+// return value says whether O must be rescaled: not when the row had seen no key
+// before (its O and sum are still zero), only when a finite reference max grows.
+__device__ __forceinline__ bool softmax_sub64(uint32_t s_tmem, int lo, int hi, float sl2, float& m_run,
+                                              float& l_run, float& alpha) {
+  if (__all_sync(0xffffffffu, hi < 0 || lo > 63)) {
+    uint32_t z[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) z[i] = 0u;
+    tmem_st32(s_tmem, z);
+    alpha = 1.0f;
+    return false;
+  }
+  float s[64];
+  {
+    uint32_t sr[64];
+    tmem_ld32_wait(s_tmem, sr);
+    tmem_ld32_wait(s_tmem + 32, sr + 32);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(sr[i]);
+  }
+  if (!__all_sync(0xffffffffu, lo <= 0 && hi >= 63)) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
+  }
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[2 * i], s[2 * i + 1]);
+#pragma unroll
+  for (int c = 16; c < 64; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+  const float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+  const float m_new = fmaxf(m_run, m_tile);
+  const bool fresh = m_run == -INFINITY;               // no key seen yet: O and l are zero
+  const bool need = !fresh && (m_new - m_run) * sl2 > 8.0f;
+  const float m_use = (need || fresh) ? m_new : m_run;
+  alpha = need ? ex2_approx((m_run - m_new) * sl2) : 1.0f;
+  const float neg = (m_use == -INFINITY) ? 0.0f : -m_use * sl2;
+  const uint64_t scale2 = f2_pack(sl2, sl2), neg2 = f2_pack(neg, neg);
+  uint64_t acc[4] = {0, 0, 0, 0};
+  uint32_t pr[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, neg2), x0, x1);
+    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+    pr[i] = pack_bf16x2(p0, p1);
+  }
+  float sum0, sum1, sum2, sum3;
+  f2_unpack(f2_add(acc[0], acc[1]), sum0, sum1);
+  f2_unpack(f2_add(acc[2], acc[3]), sum2, sum3);
+  l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
+  m_run = m_use;
+  tmem_st32(s_tmem, pr);
+  return need;
+}
+
 template <bool OUT_F32>
 __global__ void __launch_bounds__(kStreamThreads, 1)
     swa_prefill_stream_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
