@@ -17,6 +17,7 @@ built from the set definition, and hand-derived golden values.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 import threading
@@ -339,3 +340,65 @@ def swa_bwd(q, k, v, dout, window: int, n_sink: int, scale: float):
             dk[b, :, kh] += scale * (ds.T @ q[b, :, h])
             dv[b, :, kh] += p.T @ do[b, :, h]
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# The linear-attention branch of the Based hybrid ("Simple linear attention
+# language models balance the recall-throughput tradeoff", proposed method: a
+# linear attention whose feature dimension sets the recurrent state size, with no
+# position encoding, next to the sliding window).  The sink page defines linear
+# attention as a kernel approximation of softmax attention; neither page gives
+# the feature map.  Reading used: the second-order Taylor approximation of exp,
+#     kappa(q, k) = 1 + x + x^2 / 2,  x = scale * q.k   (> 0 for every x),
+# with causal normalisation
+#     out_t = sum_{s<=t} kappa(q_t, k_s) v_s / sum_{s<=t} kappa(q_t, k_s).
+# Its explicit features, phi(u) = [1, sqrt(scale) u, scale (u outer u) / sqrt(2)]
+# (F = 1 + d + d^2 entries, the outer product row-major), give kappa(q, k) =
+# phi(q).phi(k), the recurrent state S_t = sum_{s<=t} phi(k_s) v_s^T [F, dv] and
+# z_t = sum_{s<=t} phi(k_s) [F], and out_t = phi(q_t) S_t / phi(q_t).z_t.
+# ---------------------------------------------------------------------------
+
+def taylor_kernel(q, k, scale: float) -> np.ndarray:
+    """kappa(q_i, k_j) = 1 + x + x^2/2 with x = scale q_i.k_j, for q [n, d], k [m, d]."""
+    x = scale * (_f64(q) @ _f64(k).T)
+    return 1.0 + x + 0.5 * x * x
+
+
+def taylor_features(u, scale: float) -> np.ndarray:
+    """phi(u) for rows u [..., d]: [1, sqrt(scale) u, scale vec(u u^T) / sqrt(2)], float64."""
+    u = _f64(u)
+    d = u.shape[-1]
+    outer = (u[..., :, None] * u[..., None, :]).reshape(u.shape[:-1] + (d * d,))
+    one = np.ones(u.shape[:-1] + (1,))
+    return np.concatenate([one, math.sqrt(scale) * u, scale * outer / math.sqrt(2.0)], axis=-1)
+
+
+def based_linear_fwd(q, k, v, scale: float) -> np.ndarray:
+    """Causal Taylor linear attention: q, k [B, L, H, d], v [B, L, H, dv] -> out [B, L, H, dv]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, L, H, _ = q.shape
+    out = np.zeros(v.shape[:3] + (v.shape[3],))
+    causal = np.tril(np.ones((L, L), dtype=bool))
+    for b in range(B):
+        for h in range(H):
+            a = np.where(causal, taylor_kernel(q[b, :, h], k[b, :, h], scale), 0.0)
+            out[b, :, h] = (a @ v[b, :, h]) / a.sum(axis=1, keepdims=True)
+    return out
+
+
+def based_linear_state(k, v, scale: float):
+    """State after positions 0..L-1: S [B, H, F, dv] and z [B, H, F] (float64)."""
+    fk = taylor_features(k, scale)                                  # [B, L, H, F]
+    S = np.einsum("blhf,blhc->bhfc", fk, _f64(v))
+    z = fk.sum(axis=1)
+    return S, z
+
+
+def based_linear_decode(q, k, v, S, z, scale: float):
+    """One recurrent step for q, k [B, H, d], v [B, H, dv] and the state before it:
+    returns out [B, H, dv] and the new state (the token attends to itself)."""
+    fk, fq = taylor_features(k, scale), taylor_features(q, scale)   # [B, H, F]
+    S = _f64(S) + fk[..., :, None] * _f64(v)[..., None, :]
+    z = _f64(z) + fk
+    out = np.einsum("bhf,bhfc->bhc", fq, S) / np.einsum("bhf,bhf->bh", fq, z)[..., None]
+    return out, S, z
