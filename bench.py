@@ -13,7 +13,9 @@ same way: the 8B-shaped GQA prefill and the packed long-context prefill
 tokens/s against the HBM roofline), the same decode with the rotary encoding
 fused into append and decode, the rotary encoding of the GQA prefill's q and k,
 the Hadamard output projection of the GQA prefill's output (HBM GB/s), and the
-backward pass of the Based-shaped and (at L=8192) the 8B-shaped prefill.
+backward pass of the Based-shaped and (at L=8192) the 8B-shaped prefill, and
+the Based hybrid's linear-attention branch (prefill in TFLOP/s of the recurrent
+form's FLOPs, and its recurrent decode step in HBM GB/s).
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -481,6 +483,163 @@ def bench_rope_qk(name, steps, warmup, dev, flush, peaks, sampler):
     }
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP at the 1965 MHz maximum SM clock
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def based_linear_flops(w, tokens: int) -> float:
+    """Algorithmic FLOPs of the linear branch: the recurrent form's 4 F (dv + 1) per token and
+    head (adding phi(k) [v; 1]^T to the state, reading phi(q) against it)."""
+    return 4.0 * w.F * (w.dv + 1) * tokens * w.H
+
+
+def bench_based_linear(name, steps, warmup, dev, flush, peaks, sampler):
+    """Prefill of the Based linear branch: out [B, L, H, dv] and the final state."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    w = wl.LINEAR_WORKLOADS[name]
+    q, k, v = wl.make_based_linear(w, device=dev)
+    out = torch.empty(w.B, w.L, w.H, w.dv, device=dev, dtype=torch.bfloat16)
+    S = torch.empty(w.B, w.H, w.F, w.dv, device=dev)
+    z = torch.empty(w.B, w.H, w.F, device=dev)
+
+    def run(qq=q, kk=k, vv=v):
+        swa.swa_based_linear_fwd(qq, kk, vv, out, S, z, w.scale)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    flops = based_linear_flops(w, w.B * w.L)
+    tf = flops / (ms * 1e-3) / 1e12
+
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+
+    def e2e_step():
+        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv)):
+            d_.copy_(h_, non_blocking=True)
+        run(dq, dk, dv)
+        ho.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(3, steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    roof = {"bound": "alu", "achieved": round(tf, 3), "peak": round(FP32_FMA_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+            "frac": round(tf / FP32_FMA_PEAK_TFLOPS, 4),
+            "peak_source": "fp32 FMA issue rate of the CUDA cores at the maximum SM clock (derived)",
+            "traffic": profiled_traffic(name), "algorithmic_flops_per_launch": flops}
+    return {
+        "config": w.describe(), "value": round(tf, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+        "tokens_per_s": round(w.B * w.L / (ms * 1e-3), 1), "roofline": roof,
+        "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
+def bench_based_linear_decode(name, steps, warmup, dev, flush, peaks, sampler):
+    """One recurrent decode step of the linear branch for a batch: reads and writes the fp32
+    state (HBM-bound; the state of B=64 x H=16 heads is 72.7 MB, so L2 is flushed between steps)."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    w = wl.LINEAR_WORKLOADS["based_linear"]
+    B = 64
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.SEED)
+    S = torch.randn(B, w.H, w.F, w.dv, generator=g, device=dev)
+    z = 100.0 + torch.rand(B, w.H, w.F, generator=g, device=dev)
+    q = torch.randn(B, w.H, w.dk, generator=g, device=dev).bfloat16()
+    k = torch.randn(B, w.H, w.dk, generator=g, device=dev).bfloat16()
+    v = torch.randn(B, w.H, w.dv, generator=g, device=dev).bfloat16()
+    out = torch.empty(B, w.H, w.dv, device=dev, dtype=torch.bfloat16)
+
+    def run():
+        swa.swa_based_linear_decode(q, k, v, S, z, out, w.scale)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for _ in range(steps):
+            flush.fill_(1)
+            timer(run)
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    alg_bytes = B * w.H * (2 * 4 * w.F * (w.dv + 1) + 2 * (2 * w.dk + w.dv) + 2 * w.dv)
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        run()
+        ho.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(3, steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        flush.fill_(1)
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "traffic": profiled_traffic(name), "algorithmic_bytes_per_launch": alg_bytes}
+    return {
+        "config": {"workload": name, "kind": "based_linear_decode", "B": B, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "features": w.F, "state_dtype": "f32"},
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
+        "tokens_per_s": round(B / (ms * 1e-3), 1), "roofline": roof,
+        "e2e": {"value": round(alg_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "note": "includes an L2 flush per step",
+                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
 def bench_bwd(name, steps, warmup, dev, flush, peaks, sampler):
     """Backward pass (dq, dk, dv) of a prefill workload; FLOPs: five products of 2*d per
     visible pair and query head (S, dP, dV, dK, dQ), i.e. 2.5x the forward's."""
@@ -733,6 +892,20 @@ def profile_case(args):
         if swa.swa_device_error() != 0:
             raise SystemExit("device wait timed out")
         return
+    if args.profile_case in ("based_linear", "based_linear_decode"):
+        w = wl.LINEAR_WORKLOADS["based_linear"]
+        q, k, v = wl.make_based_linear(w, device=dev, B=args.B, L=args.L)
+        S = torch.zeros(q.shape[0], w.H, w.F, w.dv, device=dev)
+        z = torch.zeros(q.shape[0], w.H, w.F, device=dev)
+        out = torch.empty(q.shape[:3] + (w.dv,), device=dev, dtype=torch.bfloat16)
+        for _ in range(n):
+            if args.profile_case == "based_linear":
+                swa.swa_based_linear_fwd(q, k, v, out, S, z, w.scale)
+            else:
+                swa.swa_based_linear_decode(q[:, 0].contiguous(), k[:, 0].contiguous(), v[:, 0].contiguous(),
+                                            S, z, out[:, 0].contiguous(), w.scale)
+        torch.cuda.synchronize()
+        return
     if args.profile_case in wl.ROPE_WORKLOADS:
         c = wl.ROPE_WORKLOADS[args.profile_case]
         T = args.L or c["T"]
@@ -791,7 +964,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
     ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj,"
-                    "bwd_based_local,bwd_gqa8b_L8192")
+                    "bwd_based_local,bwd_gqa8b_L8192,based_linear,based_linear_decode")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -845,6 +1018,10 @@ def main():
             results[n] = bench_rope_qk(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         elif n == "hadamard_proj":
             results[n] = bench_hadamard(n, args.steps, args.warmup, dev, flush, peaks, sampler)
+        elif n == "based_linear":
+            results[n] = bench_based_linear(n, args.steps, args.warmup, dev, flush, peaks, sampler)
+        elif n == "based_linear_decode":
+            results[n] = bench_based_linear_decode(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         else:
             results[n] = bench_prefill(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         torch.cuda.empty_cache()

@@ -225,6 +225,33 @@ int swa_decode_rope(const void* q, const void* kcache, const void* vcache, const
                     void* workspace, size_t workspace_bytes, swa_stream_t stream);
 
 /*
+ * The linear-attention branch of the Based hybrid ("Simple linear attention
+ * language models balance the recall-throughput tradeoff", proposed method: a
+ * linear attention whose feature dimension sets the recurrent state, no
+ * position encoding).  The pages give no feature map; reading used: the
+ * second-order Taylor kernel of exp, kappa(q, k) = 1 + x + x^2/2 with
+ * x = scale q.k, i.e. features phi(u) = [1, sqrt(scale) u, scale vec(u u^T)/sqrt(2)]
+ * (F = 1 + dk + dk^2 entries, the outer product row-major), and causal
+ * normalisation: out_t = sum_{s<=t} kappa(q_t,k_s) v_s / sum_{s<=t} kappa(q_t,k_s).
+ * The recurrent state is S = sum phi(k_s) v_s^T [F, dv] and z = sum phi(k_s) [F].
+ * Supported: dk = 16, dv = 64; fp32 arithmetic.
+ *
+ * swa_based_linear_state_features(dk) = F.
+ * swa_based_linear_fwd: q, k [B, L, H, dk], v [B, L, H, dv] bf16 (read);
+ *   out [B, L, H, dv] bf16 or float32 (out_dtype SWA_DTYPE_BF16 / SWA_DTYPE_F32);
+ *   state [B, H, F, dv] and zsum [B, H, F] float32: both NULL, or both written
+ *   with the state after position L-1 (to continue with swa_based_linear_decode).
+ * swa_based_linear_decode: one generated token per sequence: q, k [B, H, dk],
+ *   v [B, H, dv] bf16; state and zsum are updated in place with the token
+ *   (S += phi(k) v^T, z += phi(k)) and out [B, H, dv] = phi(q) S / phi(q).z.
+ */
+int swa_based_linear_state_features(int dk);
+int swa_based_linear_fwd(const void* q, const void* k, const void* v, void* out, float* state, float* zsum,
+                         int B, int L, int H, int dk, int dv, float scale, int out_dtype, swa_stream_t stream);
+int swa_based_linear_decode(const void* q, const void* k, const void* v, float* state, float* zsum, void* out,
+                            int B, int H, int dk, int dv, float scale, int out_dtype, swa_stream_t stream);
+
+/*
  * Hadamard output projection, the step after attention ("Rethinking Attention
  * Output Projection: Structured Hadamard Transforms for Efficient Transformers",
  * section 2): per row, z = alpha * (y H) + beta, where H is the fixed Walsh-

@@ -37,6 +37,7 @@ EXPORTS = (
     "swa_decode_workspace_bytes", "swa_decode", "swa_status_string", "swa_device_error",
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
     "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope", "swa_bwd",
+    "swa_based_linear_state_features", "swa_based_linear_fwd", "swa_based_linear_decode",
 )
 
 _lib = None
@@ -70,6 +71,9 @@ def _load():
     lib.swa_rope_cache_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P]
     lib.swa_decode_rope.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, D, P, SZ, P]
     lib.swa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+    lib.swa_based_linear_state_features.argtypes = [I]
+    lib.swa_based_linear_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.swa_based_linear_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
@@ -78,7 +82,8 @@ def _load():
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
-                 "swa_decode_rope", "swa_bwd",
+                 "swa_decode_rope", "swa_bwd", "swa_based_linear_state_features", "swa_based_linear_fwd",
+                 "swa_based_linear_decode",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -266,6 +271,39 @@ def swa_bwd(q, k, v, out, dout, lse, dq, dk, dv, window: int, n_sink: int, scale
     st = _load().swa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                          _ptr(dv), B, Hq, Hkv, L, d, int(window), int(n_sink), _scale(scale, d), _stream(stream))
     _check(st, "swa_bwd")
+
+
+def swa_based_linear_state_features(dk: int) -> int:
+    return int(_load().swa_based_linear_state_features(int(dk)))
+
+
+def swa_based_linear_fwd(q, k, v, out, state=None, zsum=None, scale=None, stream=None) -> None:
+    """Causal Taylor linear attention: q, k [B, L, H, dk], v [B, L, H, dv] bf16 -> out (bf16 or
+    float32); state [B, H, F, dv] / zsum [B, H, F] float32, if given, receive the final state."""
+    import torch
+    B, L, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t.dtype == torch.bfloat16 and t.is_contiguous(), f"{n} bf16 contiguous")
+    _need((state is None) == (zsum is None), "state and zsum together")
+    code = SWA_DTYPE_F32 if out.dtype == torch.float32 else SWA_DTYPE_BF16
+    st = _load().swa_based_linear_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(zsum), B, L, H, dk, dv,
+                                      ctypes.c_float(scale if scale is not None else 1.0 / math.sqrt(dk)), code,
+                                      _stream(stream))
+    _check(st, "swa_based_linear_fwd")
+
+
+def swa_based_linear_decode(q, k, v, state, zsum, out, scale=None, stream=None) -> None:
+    """One token per sequence: q, k [B, H, dk], v [B, H, dv] bf16; state/zsum float32 updated
+    in place; out [B, H, dv]."""
+    import torch
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    code = SWA_DTYPE_F32 if out.dtype == torch.float32 else SWA_DTYPE_BF16
+    st = _load().swa_based_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(zsum), _ptr(out), B, H, dk, dv,
+                                         ctypes.c_float(scale if scale is not None else 1.0 / math.sqrt(dk)), code,
+                                         _stream(stream))
+    _check(st, "swa_based_linear_decode")
 
 
 def swa_hadamard_proj(y, alpha, beta, z, stream=None) -> None:

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/swa.h"
+#include "based_linear.h"
 #include "swa_internal.h"
 
 namespace {
@@ -406,6 +407,36 @@ int swa_bwd(const void* q, const void* k, const void* v, const void* out, const 
   ba.dk = dk;
   ba.dv = dv;
   cudaError_t e = swa::launch_bwd(ba, tq, tk, tv, tdo, d, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_based_linear_state_features(int dk) { return dk > 0 ? swa::based_linear_features(dk) : 0; }
+
+int swa_based_linear_fwd(const void* q, const void* k, const void* v, void* out, float* state, float* zsum,
+                         int B, int L, int H, int dk, int dv, float scale, int out_dtype, swa_stream_t stream) {
+  if (B < 0 || L < 0 || H <= 0 || !(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (out_dtype != SWA_DTYPE_BF16 && out_dtype != SWA_DTYPE_F32) return SWA_ERR_INVALID_ARG;
+  if (dk != 16 || dv != 64) return SWA_ERR_UNSUPPORTED;
+  if ((state == nullptr) != (zsum == nullptr)) return SWA_ERR_INVALID_ARG;
+  // L = 0 still writes the (zero) state when one is asked for
+  if (B == 0 || (L == 0 && state == nullptr)) return SWA_OK;
+  if (L > 0 && (!q || !k || !v || !out)) return SWA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT32_MAX) return SWA_ERR_UNSUPPORTED;
+  cudaError_t e = swa::launch_based_linear_fwd(q, k, v, out, state, zsum, B, L, H, scale, out_dtype == SWA_DTYPE_F32,
+                                               reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_based_linear_decode(const void* q, const void* k, const void* v, float* state, float* zsum, void* out,
+                            int B, int H, int dk, int dv, float scale, int out_dtype, swa_stream_t stream) {
+  if (B < 0 || H <= 0 || !(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (out_dtype != SWA_DTYPE_BF16 && out_dtype != SWA_DTYPE_F32) return SWA_ERR_INVALID_ARG;
+  if (dk != 16 || dv != 64) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!q || !k || !v || !state || !zsum || !out) return SWA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT32_MAX) return SWA_ERR_UNSUPPORTED;
+  cudaError_t e = swa::launch_based_linear_decode(q, k, v, state, zsum, out, B, H, scale, out_dtype == SWA_DTYPE_F32,
+                                                  reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

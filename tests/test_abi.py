@@ -89,3 +89,26 @@ def test_rope_and_hadamard_argument_checks(lib):
     assert lib.swa_hadamard_proj(None, None, None, None, 4, 64, 2, None) == swa.SWA_ERR_INVALID_ARG
     assert lib.swa_hadamard_proj(None, None, None, None, 0, 64, 0, None) == swa.SWA_OK
     assert lib.swa_hadamard_proj(None, None, None, None, 4, 64, 0, None) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_based_linear_argument_checks(lib):
+    F = ctypes.c_float
+    fwd = lambda **kw: lib.swa_based_linear_fwd(None, None, None, None, kw.get("state"), kw.get("zsum"),
+                                                kw.get("B", 1), kw.get("L", 8), kw.get("H", 2), kw.get("dk", 16),
+                                                kw.get("dv", 64), F(kw.get("scale", 0.25)), kw.get("dtype", 0), None)
+    assert lib.swa_based_linear_state_features(16) == 273
+    assert fwd(dk=32) == swa.SWA_ERR_UNSUPPORTED
+    assert fwd(dv=128) == swa.SWA_ERR_UNSUPPORTED
+    assert fwd(scale=0.0) == swa.SWA_ERR_INVALID_ARG
+    assert fwd(dtype=7) == swa.SWA_ERR_INVALID_ARG
+    assert fwd(H=0) == swa.SWA_ERR_INVALID_ARG
+    assert fwd() == swa.SWA_ERR_INVALID_ARG                       # null tensors
+    buf = ctypes.create_string_buffer(64)
+    assert fwd(state=ctypes.addressof(buf)) == swa.SWA_ERR_INVALID_ARG   # state without zsum
+    assert fwd(B=0) == swa.SWA_OK
+    assert fwd(L=0) == swa.SWA_OK                                 # nothing to write
+    dec = lambda **kw: lib.swa_based_linear_decode(None, None, None, None, None, None, kw.get("B", 1), 2,
+                                                   kw.get("dk", 16), 64, F(0.25), 0, None)
+    assert dec(dk=8) == swa.SWA_ERR_UNSUPPORTED
+    assert dec() == swa.SWA_ERR_INVALID_ARG
+    assert dec(B=0) == swa.SWA_OK

@@ -282,3 +282,50 @@ def make_hadamard(w: ProjWorkload, device="cpu", T: Optional[int] = None):
     alpha = 1.0 + 0.5 * _normal(g, (w.n,), device)
     beta = 0.1 * _normal(g, (w.n,), device)
     return y, alpha, beta
+
+
+@dataclasses.dataclass(frozen=True)
+class LinearWorkload:
+    """The linear-attention branch of a Based-style hybrid layer: H heads with
+    feature dimension dk (q, k) and value dimension dv, no position encoding."""
+    name: str
+    B: int
+    L: int
+    H: int
+    dk: int
+    dv: int
+    note: str = ""
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.dk)
+
+    @property
+    def F(self) -> int:
+        return 1 + self.dk + self.dk * self.dk
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "kind": "based_linear", "B": self.B, "L": self.L, "H": self.H,
+                "dk": self.dk, "dv": self.dv, "features": self.F, "dtype": "bf16"}
+
+
+LINEAR_WORKLOADS = {
+    # the linear branch next to the based_local sliding-window branch (same B, L, heads,
+    # head dim 64): feature dimension 16 gives a recurrent state of (1 + 16 + 256) x 65
+    # floats per head, about the size of the window-128 branch's 2 x 128 x 64 cache
+    "based_linear": LinearWorkload("based_linear", B=8, L=2048, H=16, dk=16, dv=64,
+                                   note="linear-attention branch of a Based-style hybrid layer"),
+}
+
+
+def make_based_linear(w: LinearWorkload, device="cpu", B: Optional[int] = None, L: Optional[int] = None,
+                      seed: int = SEED):
+    """q, k [B, L, H, dk] and v [B, L, H, dv] bf16, each N(0, 1), drawn in that order."""
+    B = w.B if B is None else B
+    L = w.L if L is None else L
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    q = _normal(g, (B, L, w.H, w.dk), device)
+    k = _normal(g, (B, L, w.H, w.dk), device)
+    v = _normal(g, (B, L, w.H, w.dv), device)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
