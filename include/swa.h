@@ -234,7 +234,12 @@ int swa_decode_rope(const void* q, const void* kcache, const void* vcache, const
  * (F = 1 + dk + dk^2 entries, the outer product row-major), and causal
  * normalisation: out_t = sum_{s<=t} kappa(q_t,k_s) v_s / sum_{s<=t} kappa(q_t,k_s).
  * The recurrent state is S = sum phi(k_s) v_s^T [F, dv] and z = sum phi(k_s) [F].
- * Supported: dk = 16, dv = 64; fp32 arithmetic.
+ * Supported: dk = 16, dv = 64.  Prefill runs on the tensor cores with bf16
+ * features, bf16 kernel values kappa within a chunk and a bf16 copy of the
+ * state as operands, fp32 accumulation; the state itself is kept in fp32.
+ * Decode is fp32 throughout.  Every pointer must be 16-byte aligned
+ * (SWA_ERR_INVALID_ARG otherwise); tensors are contiguous.  A device-side wait
+ * that runs out sets SWA_ERR_DEVICE_TIMEOUT (read with swa_device_error).
  *
  * swa_based_linear_state_features(dk) = F.
  * swa_based_linear_fwd: q, k [B, L, H, dk], v [B, L, H, dv] bf16 (read);

@@ -420,10 +420,29 @@ int swa_based_linear_fwd(const void* q, const void* k, const void* v, void* out,
   if ((state == nullptr) != (zsum == nullptr)) return SWA_ERR_INVALID_ARG;
   // L = 0 still writes the (zero) state when one is asked for
   if (B == 0 || (L == 0 && state == nullptr)) return SWA_OK;
-  if (L > 0 && (!q || !k || !v || !out)) return SWA_ERR_INVALID_ARG;
+  if (L > 0 && (!q || !k || !v || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+    return SWA_ERR_INVALID_ARG;
+  if (state != nullptr && !aligned16(state)) return SWA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT32_MAX) return SWA_ERR_UNSUPPORTED;
-  cudaError_t e = swa::launch_based_linear_fwd(q, k, v, out, state, zsum, B, L, H, scale, out_dtype == SWA_DTYPE_F32,
-                                               reinterpret_cast<cudaStream_t>(stream));
+  DeviceInfo* di = nullptr;
+  const int st = device_info(&di);
+  if (st != SWA_OK) return st;
+  swa::BasedLinearArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.state = state;
+  a.zsum = zsum;
+  a.B = B;
+  a.L = L;
+  a.H = H;
+  a.scale = scale;
+  a.out_f32 = out_dtype == SWA_DTYPE_F32 ? 1 : 0;
+  a.timeout_ns = g_timeout_ns.load();
+  a.debug_flags = g_debug_flags.load();
+  a.err = di->err;
+  cudaError_t e = swa::launch_based_linear_fwd(a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -433,7 +452,7 @@ int swa_based_linear_decode(const void* q, const void* k, const void* v, float* 
   if (out_dtype != SWA_DTYPE_BF16 && out_dtype != SWA_DTYPE_F32) return SWA_ERR_INVALID_ARG;
   if (dk != 16 || dv != 64) return SWA_ERR_UNSUPPORTED;
   if (B == 0) return SWA_OK;
-  if (!q || !k || !v || !state || !zsum || !out) return SWA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !state || !zsum || !out || !aligned16(state)) return SWA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT32_MAX) return SWA_ERR_UNSUPPORTED;
   cudaError_t e = swa::launch_based_linear_decode(q, k, v, state, zsum, out, B, H, scale, out_dtype == SWA_DTYPE_F32,
                                                   reinterpret_cast<cudaStream_t>(stream));

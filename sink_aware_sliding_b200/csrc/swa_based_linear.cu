@@ -9,13 +9,13 @@
 // (F = 1 + dk + dk^2, the outer product row-major), state S = sum phi(k) v^T
 // [F, dv] and z = sum phi(k) [F], and out_t = phi(q_t) S_t / phi(q_t).z_t.
 //
-// First version, fp32 on the CUDA cores, dk = 16 and dv = 64 (F = 273): one CTA
-// per (sequence, head).  The state lives in registers, spread over 4 x 65
-// threads: thread (c, g) holds column c of S (c = 64: z, i.e. v = 1) for the
-// feature range g.  Prefill walks the sequence in chunks of 64 tokens: the
-// output of a chunk is phi(Q) S (the earlier chunks, from the state) plus the
-// causal kappa(Q K^T) V of the chunk itself; then S += phi(K)^T V.  Decode is one
-// such step for one token, reading and writing the state in global memory.
+// dk = 16 and dv = 64 (F = 273).  Prefill walks each (sequence, head) in
+// chunks: the output of a chunk is phi(Q) S (the earlier chunks, from the state)
+// plus the causal kappa(Q K^T) V of the chunk itself, normalised by the same
+// two terms with v replaced by 1; then S += phi(K)^T V.  The tensor-core kernel
+// (swa_based_linear_tc.cu) does this with tcgen05; this file holds the CUDA-core
+// form of the same chunked step (fp32 throughout) and the decode step, which
+// reads and writes the state in global memory.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,7 +47,7 @@ __device__ __forceinline__ float feature(const float* u, int f, float rs, float 
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    swa_based_linear_fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    swa_based_linear_fwd_simt_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                 const __nv_bfloat16* __restrict__ v, void* __restrict__ out, float* __restrict__ state,
                                 float* __restrict__ zsum, int L, int H, float scale, int out_f32) {
   extern __shared__ float sm[];
@@ -151,11 +151,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // One decode step per (sequence, head): S += phi(k) v^T, z += phi(k), out = phi(q) S / phi(q).z.
-__global__ void __launch_bounds__(kThreads)
+// 256 threads: thread (c4, g) owns columns 4 c4 .. 4 c4 + 3 of S for the features
+// f = g, g + 16, ...; the loads of a thread's rows are issued in batches so that
+// several 16-byte reads are in flight per thread (the step is HBM-bound).
+constexpr int kDecThreads = 256;
+constexpr int kDecGroups = kDecThreads / (kDV / 4);        // 16
+constexpr int kDecRows = (kF + kDecGroups - 1) / kDecGroups;  // 18 rows per group at most
+
+__global__ void __launch_bounds__(kDecThreads)
     swa_based_linear_decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                    const __nv_bfloat16* __restrict__ v, float* __restrict__ state,
                                    float* __restrict__ zsum, void* __restrict__ out, int H, float scale, int out_f32) {
-  __shared__ float qs[kDK], ks[kDK], vs[kCols], fq[kF], fk[kF], part[kGroups][kCols];
+  __shared__ float qs[kDK], ks[kDK], fq[kF], fk[kF];
+  __shared__ float4 part[kDecGroups][kDV / 4];
+  __shared__ float zpart[kDecThreads / 32];
   const long long bh = blockIdx.x;
   const int tid = threadIdx.x;
   const float rs = sqrtf(scale), s_over_r2 = scale * 0.70710678118654752f;
@@ -163,29 +172,67 @@ __global__ void __launch_bounds__(kThreads)
     qs[tid] = bf16_at(q, bh * kDK + tid);
     ks[tid] = bf16_at(k, bh * kDK + tid);
   }
-  if (tid < kCols) vs[tid] = tid == kDV ? 1.f : bf16_at(v, bh * kDV + tid);
+  const int c4 = tid % (kDV / 4), g = tid / (kDV / 4);
+  float4 vv;
+  {
+    const __nv_bfloat16* pv = v + bh * kDV + 4 * c4;
+    vv = make_float4(__bfloat162float(pv[0]), __bfloat162float(pv[1]), __bfloat162float(pv[2]),
+                     __bfloat162float(pv[3]));
+  }
   __syncthreads();
-  for (int f = tid; f < kF; f += kThreads) {
+  for (int f = tid; f < kF; f += kDecThreads) {
     fq[f] = feature(qs, f, rs, s_over_r2);
     fk[f] = feature(ks, f, rs, s_over_r2);
   }
   __syncthreads();
-  if (tid < kGroups * kCols) {
-    const int c = tid % kCols, g = tid / kCols;
-    const int f0 = g * kFPer, f1 = min(kF, f0 + kFPer);
-    float acc = 0.f;
-    for (int f = f0; f < f1; ++f) {
-      float* p = c < kDV ? state + (bh * kF + f) * kDV + c : zsum + bh * kF + f;
-      const float s_new = fmaf(fk[f], vs[c], *p);
-      *p = s_new;
-      acc = fmaf(fq[f], s_new, acc);
-    }
-    part[g][c] = acc;
+  float4* S4 = reinterpret_cast<float4*>(state + bh * kF * kDV) + c4;
+  float4 row[kDecRows];
+#pragma unroll
+  for (int i = 0; i < kDecRows; ++i) {
+    const int f = g + kDecGroups * i;
+    if (f < kF) row[i] = S4[f * (kDV / 4)];
   }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < kDecRows; ++i) {
+    const int f = g + kDecGroups * i;
+    if (f < kF) {
+      const float a = fk[f], b = fq[f];
+      float4 r = row[i];
+      r.x = fmaf(a, vv.x, r.x);
+      r.y = fmaf(a, vv.y, r.y);
+      r.z = fmaf(a, vv.z, r.z);
+      r.w = fmaf(a, vv.w, r.w);
+      S4[f * (kDV / 4)] = r;
+      acc.x = fmaf(b, r.x, acc.x);
+      acc.y = fmaf(b, r.y, acc.y);
+      acc.z = fmaf(b, r.z, acc.z);
+      acc.w = fmaf(b, r.w, acc.w);
+    }
+  }
+  part[g][c4] = acc;
+  // normaliser: z += phi(k), den = phi(q).z
+  float zd = 0.f;
+  for (int f = tid; f < kF; f += kDecThreads) {
+    const float zn = zsum[bh * kF + f] + fk[f];
+    zsum[bh * kF + f] = zn;
+    zd = fmaf(fq[f], zn, zd);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zd += __shfl_xor_sync(0xffffffffu, zd, o);
+  if ((tid & 31) == 0) zpart[tid >> 5] = zd;
   __syncthreads();
   if (tid < kDV) {
-    const float num = part[0][tid] + part[1][tid] + part[2][tid] + part[3][tid];
-    const float den = part[0][kDV] + part[1][kDV] + part[2][kDV] + part[3][kDV];
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < kDecThreads / 32; ++i) den += zpart[i];
+    float num = 0.f;
+    const int cc = tid >> 2, e = tid & 3;
+#pragma unroll
+    for (int i = 0; i < kDecGroups; ++i) {
+      const float4 p = part[i][cc];
+      num += e == 0 ? p.x : (e == 1 ? p.y : (e == 2 ? p.z : p.w));
+    }
     const long long idx = bh * kDV + tid;
     if (out_f32) static_cast<float*>(out)[idx] = num / den;
     else static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(num / den);
@@ -196,23 +243,21 @@ __global__ void __launch_bounds__(kThreads)
 
 int based_linear_features(int dk) { return 1 + dk + dk * dk; }
 
-cudaError_t launch_based_linear_fwd(const void* q, const void* k, const void* v, void* out, float* state,
-                                    float* zsum, int B, int L, int H, float scale, bool out_f32,
-                                    cudaStream_t stream) {
+cudaError_t launch_based_linear_fwd_simt(const BasedLinearArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(float) * (2 * kChunk * kDK + kChunk * kCols + kChunk * kF +
                                        kGroups * kChunk * kCols + kChunk * kChunk);
-  cudaError_t e = cudaFuncSetAttribute(swa_based_linear_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(swa_based_linear_fwd_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  swa_based_linear_fwd_kernel<<<B * H, kThreads, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), out, state, zsum, L, H, scale, out_f32 ? 1 : 0);
+  swa_based_linear_fwd_simt_kernel<<<a.B * a.H, kThreads, smem, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), a.out, a.state, a.zsum, a.L, a.H, a.scale, a.out_f32);
   return cudaGetLastError();
 }
 
 cudaError_t launch_based_linear_decode(const void* q, const void* k, const void* v, float* state, float* zsum,
                                        void* out, int B, int H, float scale, bool out_f32, cudaStream_t stream) {
-  swa_based_linear_decode_kernel<<<B * H, kThreads, 0, stream>>>(
+  swa_based_linear_decode_kernel<<<B * H, kDecThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), state, zsum, out, H, scale, out_f32 ? 1 : 0);
   return cudaGetLastError();
