@@ -4,23 +4,32 @@
 // attention language models balance the recall-throughput tradeoff", proposed
 // method): out_t = phi(q_t) S_t / phi(q_t).z_t with S_t = sum_{s<=t} phi(k_s) v_s^T.
 //
+// The quadratic part of phi(q).phi(k) = 1 + x + x^2/2 is symmetric in the pair
+// (a, b), so the kernel uses the 136 products with a <= b instead of all 256:
+// u_a^2 with weight scale/sqrt(2) and u_a u_b (a < b) with weight scale, whose
+// dot products give the same kernel.  Internal feature order: the 16 linear
+// terms sqrt(scale) u, the constant 1, the 136 products (a-major), zeros up to
+// 192 columns; 153 are real.  The state is returned in the interface order
+// [1, linear, all 256 products], an off-diagonal internal row split back as
+// row / sqrt(2) into (a, b) and (b, a).
+//
 // One CTA per (sequence, head) walks the sequence in chunks of 128 tokens.  With
-// V1 = [V | 1 | 0...] (80 columns: the values, a column of ones that turns the
-// same products into the normaliser, zero padding) a chunk is
-//   X  = phi_lin(Q) phi_lin(K)^T                       (= scale q.k, K = 16)
-//   O  = phi(Q) S_bf16  +  kappa_causal(X) V1           (S from earlier chunks)
-//   S += phi(K)^T V1
-// where kappa(x) = 1 + x + x^2/2 with the causal mask applied, and out = O[:, :64]
-// / O[:, 64].  Features are kept in an internal order: the 256 products
-// u_a u_b (a-major), then the 16 linear terms, then the constant, then zeros up to
-// 384 = 3 x 128 feature rows, so that S is three 128-row accumulators.
+// V1 = [V | 1 | 0...] (the values, a column of ones that turns the same products
+// into the normaliser, zero padding) a chunk is
+//   X   = phi_lin(Q) phi_lin(K)^T                  (= scale q.k; K = 16)
+//   O   = phi(Q) S_bf16 + kappa_causal(X) V1        (S from the earlier chunks)
+//   S^T += V1^T phi(K)                              (M = value column, N = 192 features)
+// with kappa(x) = 1 + x + x^2/2 under the causal mask and out = O[:, :64] / O[:, 64].
+// S is accumulated transposed (tensor-memory lane = value column), so that each
+// lane's row is one row of the K-major bf16 operand of the next chunk's phi(Q) S.
+// phi(Q) and phi(K) have buffers of their own and V1 and O two each, so the
+// feature rows of the next chunk are written while this chunk's products run.
 //
 // Roles (288 threads):
-//   warps 0-3  token rows: q/k loads, phi(Q) and phi_lin(K) into shared memory,
-//              kappa of X into P (bf16, over X's own tensor-memory columns),
-//              phi(K), the output epilogue;
-//   warps 4-7  state: V loads into V1, S (tensor memory, fp32) -> S_bf16 (shared,
-//              the B operand of the next chunk), the final state;
+//   warps 0-3  token rows of the K side: k loads, phi(K), kappa(X) -> P (bf16,
+//              over X's own tensor-memory columns), the output epilogue;
+//   warps 4-7  token rows of the Q side and state lanes: q and v loads, phi(Q),
+//              V1, S^T -> S_bf16 between chunks, the final state;
 //   warp 8     one thread issues every MMA.
 // All waits on mbarriers are bounded; on a time-out the CTA stops, drains its
 // MMAs, frees its tensor memory and records the status.
@@ -29,6 +38,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <utility>
 
 #include "based_linear.h"
 #include "ptx.cuh"
@@ -39,19 +49,25 @@ namespace {
 namespace bl {
 constexpr int kChunk = 128;                  // tokens per chunk (MMA M)
 constexpr int kDK = 16, kDV = 64;
-constexpr int kF = 1 + kDK + kDK * kDK;      // 273 features
+constexpr int kF = 1 + kDK + kDK * kDK;      // 273 features in the interface order
+constexpr int kFI = 192;                     // internal feature columns (153 real)
+constexpr int kFReal = kDK + 1 + kDK * (kDK + 1) / 2;   // 153
 constexpr int kNV = 80;                      // V1 columns: 64 values, the ones column, padding
-constexpr int kQSteps = 18;                  // phi(Q) S_bf16 over features 0 .. 287 (K steps of 16)
+constexpr int kQSteps = 10;                  // phi(Q) S_bf16 over features 0 .. 159 (K steps of 16)
+constexpr int kGranules = 20;                // 16-byte granules of a feature row written per chunk (0 .. 159)
 constexpr int kThreads = 288;
 constexpr int kMmaWarp = 8;
 constexpr uint32_t kCh = kChunk * 128;       // one 64-column chunk of a 128-row operand: 16 KB
 constexpr uint32_t kSbCh = kNV * 128;        // one 64-column chunk of S_bf16 (80 rows): 10 KB
-constexpr uint32_t OFF_PHI = 0;              // [128 tokens x 384 features], 6 chunks
-constexpr uint32_t OFF_KLIN = 6 * kCh;       // [128 tokens x 64]: phi_lin(K) in columns 0 .. 15
-constexpr uint32_t OFF_V1 = 7 * kCh;         // values chunk, then the ones chunk
-constexpr uint32_t OFF_SB = 9 * kCh;         // S_bf16 [80 columns of S x 384 features], 6 chunks
-constexpr uint32_t OFF_BAR = OFF_SB + 6 * kSbCh;
-enum { B_PHIQ, B_V1, B_X, B_O1, B_P, B_PHIK, B_OFULL, B_OFREE, B_SFULL, B_SB, B_DRAIN, kNumBars };
+constexpr uint32_t OFF_PHIQ = 0;             // [128 tokens x 192 features], 3 chunks
+constexpr uint32_t OFF_PHIK = 3 * kCh;
+constexpr uint32_t OFF_V1 = 6 * kCh;         // two buffers of [values chunk | ones chunk]
+constexpr uint32_t OFF_SB = 10 * kCh;        // S_bf16 [80 value columns x 192 features], 3 chunks
+constexpr uint32_t OFF_BAR = OFF_SB + 3 * kSbCh;
+enum {
+  B_PHIQ, B_PHIK, B_V1, B_V1b, B_X, B_O1, B_P, B_OFULL, B_OFULLb, B_OFREE, B_OFREEb, B_SFULL, B_SB, B_DRAIN,
+  kNumBars
+};
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + kNumBars * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
 constexpr uint32_t kSmemUsed = OFF_ABORT + 4;
@@ -59,14 +75,32 @@ constexpr uint32_t kSmem = kSmemUsed + 1024;  // slack to align the base to 1024
 static_assert(kSmem <= 232448, "shared memory");
 // tensor-memory columns
 constexpr uint32_t T_X = 0;                  // X (fp32, 128 columns); P (bf16 pairs) over its first 64
-constexpr uint32_t T_O = 128;                // O (80 columns)
-constexpr uint32_t T_S = 256;                // S tile j at T_S + 80 j, j = 0 .. 2
+constexpr uint32_t T_O = 128;                // O buffer j at T_O + 80 j (80 columns each)
+constexpr uint32_t T_ST = 288;               // S^T: lanes = value columns, 192 feature columns
 // instruction descriptors (bf16 x bf16 -> fp32); bit 15 makes A MN-major
 constexpr uint32_t IDESC_X = make_idesc(1, 128, 128, false);
 constexpr uint32_t IDESC_QS = make_idesc(1, 128, kNV, false);
 constexpr uint32_t IDESC_PV = make_idesc(1, 128, kNV, true);
-constexpr uint32_t IDESC_KV = make_idesc(1, 128, kNV, true) | (1u << 15);
+constexpr uint32_t IDESC_KV = make_idesc(1, 128, kFI, true) | (1u << 15);
 constexpr int kStatusTimeout = 4;            // SWA_ERR_DEVICE_TIMEOUT
+
+// Product p (0 .. 135) of the symmetric pairs a <= b in a-major order.
+__host__ __device__ constexpr int pair_a(int p) {
+  int a = 0;
+  while (p >= kDK - a) {
+    p -= kDK - a;
+    ++a;
+  }
+  return a;
+}
+__host__ __device__ constexpr int pair_b(int p) {
+  int a = 0;
+  while (p >= kDK - a) {
+    p -= kDK - a;
+    ++a;
+  }
+  return a + p;
+}
 }  // namespace bl
 
 // K-major operand with 128-byte rows in 64-column chunks of `chunk` bytes: K step kk (16 columns).
@@ -110,37 +144,48 @@ __device__ __forceinline__ bool bl_wait(uint32_t bar, uint32_t parity, const BlC
     }
   }
 }
-
 // The same wait taken by a whole warp: true only if every lane's wait succeeded, so
-// that the warp-collective tensor-memory loads that follow run converged.
+// that the warp-collective tensor-memory accesses that follow run converged.
 __device__ __forceinline__ bool bl_warp_wait(uint32_t bar, uint32_t parity, const BlCtl& c) {
   const bool ok = bl_wait(bar, parity, c);
   return __all_sync(0xffffffffu, ok);
 }
 
-// Row t of phi(u) (internal order) into the K-major feature operand; `keep` = 0
-// writes a zero row (tokens past the end of the sequence).
-__device__ __forceinline__ void write_phi_row(uint32_t phi, int t, const float* u, float c2, float rs, bool keep) {
+// Internal feature f (compile-time) of u.
+template <int F>
+__device__ __forceinline__ float feat(const float* u, float rs, float c2, float s) {
   using namespace bl;
-#pragma unroll
-  for (int a = 0; a < kDK; ++a) {
-    const float ca = keep ? c2 * u[a] : 0.f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float* ub = u + 8 * h;
-      sts128(gran(phi + (a >> 2) * kCh, t, (a & 3) * 2 + h), pack_bf16x2(ca * ub[0], ca * ub[1]),
-             pack_bf16x2(ca * ub[2], ca * ub[3]), pack_bf16x2(ca * ub[4], ca * ub[5]),
-             pack_bf16x2(ca * ub[6], ca * ub[7]));
-    }
+  if constexpr (F < kDK) {
+    return rs * u[F];
+  } else if constexpr (F == kDK) {
+    return 1.0f;
+  } else if constexpr (F < kFReal) {
+    constexpr int a = pair_a(F - kDK - 1), b = pair_b(F - kDK - 1);
+    return (a == b ? c2 : s) * u[a] * u[b];
+  } else {
+    return 0.0f;
   }
-  const float r = keep ? rs : 0.f;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const float* ub = u + 8 * h;
-    sts128(gran(phi + 4 * kCh, t, h), pack_bf16x2(r * ub[0], r * ub[1]), pack_bf16x2(r * ub[2], r * ub[3]),
-           pack_bf16x2(r * ub[4], r * ub[5]), pack_bf16x2(r * ub[6], r * ub[7]));
-  }
-  sts128(gran(phi + 4 * kCh, t, 2), keep ? 0x3F80u : 0u, 0u, 0u, 0u);   // the constant feature (1.0)
+}
+template <int G>
+__device__ __forceinline__ void write_granule(uint32_t phi, int t, const float* u, float rs, float c2, float s,
+                                              float keep) {
+  constexpr int f = 8 * G;
+  sts128(gran(phi + (G >> 3) * bl::kCh, t, G & 7),
+         pack_bf16x2(keep * feat<f>(u, rs, c2, s), keep * feat<f + 1>(u, rs, c2, s)),
+         pack_bf16x2(keep * feat<f + 2>(u, rs, c2, s), keep * feat<f + 3>(u, rs, c2, s)),
+         pack_bf16x2(keep * feat<f + 4>(u, rs, c2, s), keep * feat<f + 5>(u, rs, c2, s)),
+         pack_bf16x2(keep * feat<f + 6>(u, rs, c2, s), keep * feat<f + 7>(u, rs, c2, s)));
+}
+template <int... G>
+__device__ __forceinline__ void write_granules(uint32_t phi, int t, const float* u, float rs, float c2, float s,
+                                               float keep, std::integer_sequence<int, G...>) {
+  (write_granule<G>(phi, t, u, rs, c2, s, keep), ...);
+}
+// Row t of phi(u) (internal order, features 0 .. 159) into a K-major feature operand;
+// keep = 0 writes a zero row (tokens past the end of the sequence).
+__device__ __forceinline__ void write_phi_row(uint32_t phi, int t, const float* u, float rs, float c2, float s,
+                                              bool keep) {
+  write_granules(phi, t, u, rs, c2, s, keep ? 1.0f : 0.0f, std::make_integer_sequence<int, bl::kGranules>{});
 }
 
 __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, float* u) {
@@ -152,8 +197,37 @@ __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, float
   }
 }
 
-// Internal feature row -> position in the state layout [1, linear (16), products (256)].
-__device__ __forceinline__ int abi_feature(int f) { return f < 256 ? 17 + f : (f < 272 ? 1 + (f - 256) : 0); }
+// Internal feature F of one state lane (value column n < 64, or z for n = 64) into the
+// interface layout [1, linear (16), products (256, row-major)].
+template <int F>
+__device__ __forceinline__ void store_state_feature(float val, int n, float* st, float* zs) {
+  using namespace bl;
+  if constexpr (F < kFReal) {
+    auto put = [&](int fa, float x) {
+      if (n < kDV) st[fa * kDV + n] = x;
+      else zs[fa] = x;
+    };
+    if constexpr (F < kDK) {
+      put(1 + F, val);
+    } else if constexpr (F == kDK) {
+      put(0, val);
+    } else {
+      constexpr int a = pair_a(F - kDK - 1), b = pair_b(F - kDK - 1);
+      if constexpr (a == b) {
+        put(1 + kDK + kDK * a + a, val);
+      } else {
+        const float h = val * 0.70710678118654752f;
+        put(1 + kDK + kDK * a + b, h);
+        put(1 + kDK + kDK * b + a, h);
+      }
+    }
+  }
+}
+template <int P, int... E>
+__device__ __forceinline__ void store_state_piece(const uint32_t* sr, int n, float* st, float* zs,
+                                                  std::integer_sequence<int, E...>) {
+  (store_state_feature<32 * P + E>(__uint_as_float(sr[E]), n, st, zs), ...);
+}
 
 __global__ void __launch_bounds__(bl::kThreads, 1)
     swa_based_linear_tc_kernel(const __grid_constant__ BasedLinearArgs a) {
@@ -171,17 +245,26 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int nc = (a.L + kChunk - 1) / kChunk;
 
-  // zero the feature operand (its padding stays zero), S_bf16 (features past 272
-  // stay zero) and the ones chunk of V1, then put the ones in place
-  for (uint32_t o = tid * 16; o < 6 * kCh; o += kThreads * 16) sts128(base + OFF_PHI + o, 0, 0, 0, 0);
-  for (uint32_t o = tid * 16; o < 6 * kSbCh; o += kThreads * 16) sts128(base + OFF_SB + o, 0, 0, 0, 0);
-  for (uint32_t o = tid * 16; o < kCh; o += kThreads * 16) sts128(base + OFF_V1 + kCh + o, 0, 0, 0, 0);
+  // zero both feature operands (their padding columns stay zero), S_bf16 and the
+  // ones chunks of both V1 buffers, then put the ones in place (column 64 = 1.0)
+  for (uint32_t o = tid * 16; o < 6 * kCh; o += kThreads * 16) sts128(base + OFF_PHIQ + o, 0, 0, 0, 0);
+  for (uint32_t o = tid * 16; o < 3 * kSbCh; o += kThreads * 16) sts128(base + OFF_SB + o, 0, 0, 0, 0);
+  for (uint32_t o = tid * 16; o < kCh; o += kThreads * 16) {
+    sts128(base + OFF_V1 + kCh + o, 0, 0, 0, 0);
+    sts128(base + OFF_V1 + 3 * kCh + o, 0, 0, 0, 0);
+  }
   __syncthreads();
-  if (tid < kChunk) sts32(gran(base + OFF_V1 + kCh, tid, 0), 0x3F80u);   // column 64 of V1 = 1.0
+  if (tid < kChunk) {
+    sts32(gran(base + OFF_V1 + kCh, tid, 0), 0x3F80u);
+    sts32(gran(base + OFF_V1 + 3 * kCh, tid, 0), 0x3F80u);
+  }
   fence_proxy_async_smem();
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == B_PHIQ || i == B_V1 || i == B_P || i == B_PHIK ||
-                                                          i == B_OFREE || i == B_SB) ? 128 : 1);
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool threads = i == B_PHIQ || i == B_PHIK || i == B_V1 || i == B_V1b || i == B_P || i == B_OFREE ||
+                           i == B_OFREEb || i == B_SB;
+      mbar_init(bar(i), threads ? 128 : 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -193,55 +276,40 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const float c2 = a.scale * 0.70710678118654752f, rs = sqrtf(a.scale);
+  const float sc = a.scale, c2 = a.scale * 0.70710678118654752f, rs = sqrtf(a.scale);
 
   if (warp < 4) {
-    // ---------------------------------------------------------------- token rows
+    // ---------------------------------------------------------------- K-side token rows
     const int t = tid;                                   // row of the chunk = tensor-memory lane
     const uint32_t lane_t = static_cast<uint32_t>(warp * 32) << 16;
-    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-    auto load_qk = [&](int i, uint4* r) {
+    auto load_k = [&](int i, uint4* r) {
       const int tok = i * kChunk + t;
       if (i < nc && tok < a.L) {
-        const long long row = (static_cast<long long>(b) * a.L + tok) * a.H + h;
-        const uint4* pq = reinterpret_cast<const uint4*>(qg + row * kDK);
-        const uint4* pk = reinterpret_cast<const uint4*>(kg + row * kDK);
-        r[0] = __ldg(pq);
-        r[1] = __ldg(pq + 1);
-        r[2] = __ldg(pk);
-        r[3] = __ldg(pk + 1);
+        const uint4* pk = reinterpret_cast<const uint4*>(kg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDK);
+        r[0] = __ldg(pk);
+        r[1] = __ldg(pk + 1);
       } else {
-        r[0] = r[1] = r[2] = r[3] = make_uint4(0, 0, 0, 0);
+        r[0] = r[1] = make_uint4(0, 0, 0, 0);
       }
     };
-    uint4 cur[4], nxt[4];
-    load_qk(0, cur);
+    uint4 cur[2], nxt[2];
+    load_k(0, cur);
     bool ok = true;
     for (int i = 0; i < nc && ok; ++i) {
       const int n = min(kChunk, a.L - i * kChunk);
-      load_qk(i + 1, nxt);
-      float u[16];
-      // phi(Q) and phi_lin(K) once the previous chunk's MMAs are done with the operand
+      load_k(i + 1, nxt);
+      // phi(K) once the previous chunk's products are done with the operand
       if (i > 0 && !(ok = bl_warp_wait(bar(B_SFULL), (i - 1) & 1, ctl))) break;
-      unpack16(cur[0], cur[1], u);
-      write_phi_row(base + OFF_PHI, t, u, c2, rs, true);
-      unpack16(cur[2], cur[3], u);
       {
-        const bool keep = t < n;
-        const float r = keep ? rs : 0.f;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float* ub = u + 8 * hh;
-          sts128(gran(base + OFF_KLIN, t, hh), pack_bf16x2(r * ub[0], r * ub[1]), pack_bf16x2(r * ub[2], r * ub[3]),
-                 pack_bf16x2(r * ub[4], r * ub[5]), pack_bf16x2(r * ub[6], r * ub[7]));
-        }
+        float u[16];
+        unpack16(cur[0], cur[1], u);
+        write_phi_row(base + OFF_PHIK, t, u, rs, c2, sc, t < n);
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar(B_PHIQ));
+      mbar_arrive(bar(B_PHIK));
       // kappa(X) with the causal mask -> P (bf16 pairs over X's first 64 columns)
       if (!(ok = bl_warp_wait(bar(B_X), i & 1, ctl))) break;
-      __syncwarp();
       tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -261,21 +329,16 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P));
-      // phi(K) over phi(Q) once O = phi(Q) S_bf16 has read it
-      if (!(ok = bl_warp_wait(bar(B_O1), i & 1, ctl))) break;
-      write_phi_row(base + OFF_PHI, t, u, c2, rs, t < n);
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_PHIK));
       // epilogue: out = O[:, :64] / O[:, 64]
-      if (!(ok = bl_warp_wait(bar(B_OFULL), i & 1, ctl))) break;
-      __syncwarp();
+      const int ob = i & 1;
+      if (!(ok = bl_warp_wait(bar(B_OFULL + ob), (i >> 1) & 1, ctl))) break;
       tc_fence_after();
       uint32_t orr[96];
-      tmem_ld32_wait(tmem + lane_t + T_O, orr);
-      tmem_ld32_wait(tmem + lane_t + T_O + 32, orr + 32);
-      tmem_ld32_wait(tmem + lane_t + T_O + 64, orr + 64);
+      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob, orr);
+      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob + 32, orr + 32);
+      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob + 64, orr + 64);
       tc_fence_before();
-      mbar_arrive(bar(B_OFREE));
+      mbar_arrive(bar(B_OFREE + ob));
       if (t < n) {
         const float inv = 1.0f / __uint_as_float(orr[64]);
         const long long row = (static_cast<long long>(b) * a.L + i * kChunk + t) * a.H + h;
@@ -297,68 +360,90 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+      cur[0] = nxt[0];
+      cur[1] = nxt[1];
     }
   } else if (warp < 8) {
-    // ---------------------------------------------------------------- state
-    const int r = tid - 128;                             // token row for V loads
+    // ---------------------------------------------------------------- Q-side token rows, state lanes
+    const int r = tid - 128;                             // token row (phi(Q), V1) and state lane
     const int w = warp - 4;                              // tensor-memory lane quarter
     const uint32_t lane_t = static_cast<uint32_t>(w * 32) << 16;
+    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
-    auto load_v = [&](int i, uint4* dst) {
+    auto load_qv = [&](int i, uint4* qr, uint4* vr) {
       const int tok = i * kChunk + r;
       if (i < nc && tok < a.L) {
-        const uint4* pv = reinterpret_cast<const uint4*>(
-            vg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDV);
+        const long long row = (static_cast<long long>(b) * a.L + tok) * a.H + h;
+        const uint4* pq = reinterpret_cast<const uint4*>(qg + row * kDK);
+        const uint4* pv = reinterpret_cast<const uint4*>(vg + row * kDV);
+        qr[0] = __ldg(pq);
+        qr[1] = __ldg(pq + 1);
 #pragma unroll
-        for (int g = 0; g < 8; ++g) dst[g] = __ldg(pv + g);
+        for (int g = 0; g < 8; ++g) vr[g] = __ldg(pv + g);
       } else {
+        qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int g = 0; g < 8; ++g) dst[g] = make_uint4(0, 0, 0, 0);
+        for (int g = 0; g < 8; ++g) vr[g] = make_uint4(0, 0, 0, 0);
       }
     };
-    uint4 vr[8];
-    load_v(0, vr);
+    // chunk c's values into V1 buffer c & 1 and phi(Q) of chunk c
+    auto put_v = [&](int c, const uint4* vr) {
+      const uint32_t vb = base + OFF_V1 + (c & 1) * 2 * kCh;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) sts128(gran(vb, r, g), vr[g].x, vr[g].y, vr[g].z, vr[g].w);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_V1 + (c & 1)));
+    };
+    auto put_q = [&](const uint4* qr) {
+      float u[16];
+      unpack16(qr[0], qr[1], u);
+      write_phi_row(base + OFF_PHIQ, r, u, rs, c2, sc, true);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_PHIQ));
+    };
+    uint4 qr[2], vr[8];
     bool ok = true;
+    if (nc > 0) {
+      load_qv(0, qr, vr);
+      put_v(0, vr);
+      put_q(qr);
+      load_qv(1, qr, vr);
+    }
     for (int i = 0; i < nc && ok; ++i) {
       if (i > 0) {
+        // S^T after chunk i-1 -> S_bf16 (row n = value column, K-major over the features)
         if (!(ok = bl_warp_wait(bar(B_SFULL), (i - 1) & 1, ctl))) break;
-        __syncwarp();
         tc_fence_after();
-      }
-      // this chunk's values into V1 (the previous chunk's MMAs are done with it)
+        if (w < 3) {
+          const int n = 32 * w + lane;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) sts128(gran(base + OFF_V1, r, g), vr[g].x, vr[g].y, vr[g].z, vr[g].w);
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_V1));
-      load_v(i + 1, vr);
-      if (i > 0) {
-        // S after chunk i-1 -> S_bf16, the K-major B operand [80 x 384] of phi(Q) S:
-        // thread = feature row f; lanes f, f^1 swap values so that each stores a pair
-        const bool odd = lane & 1;
-#pragma unroll 1
-        for (int j = 0; j < 3; ++j) {
-          if (j == 2 && w > 0) break;                    // features 288 .. 383 are zero
-          const int f = 128 * j + 32 * w + lane;
-          uint32_t sr[96];
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j, sr);
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j + 32, sr + 32);
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j + 64, sr + 64);
-          const int fe = (f & ~1) & 63;                  // even feature of the pair, within its chunk
-          const uint32_t cb = base + OFF_SB + (f >> 6) * kSbCh;
+          for (int p = 0; p < 5; ++p) {
+            uint32_t sr[32];
+            tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
+            if (n < kNV) {
 #pragma unroll
-          for (int m = 0; m < kNV / 2; ++m) {
-            const float mine0 = __uint_as_float(sr[2 * m]), mine1 = __uint_as_float(sr[2 * m + 1]);
-            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
-            const int row = 2 * m + (odd ? 1 : 0);
-            const uint32_t val = odd ? pack_bf16x2(other, mine1) : pack_bf16x2(mine0, other);
-            sts32(cb + row * 128 + ((((fe >> 3) ^ row) & 7) << 4) + (fe & 7) * 2, val);
+              for (int g = 0; g < 4; ++g) {
+                const int G = 4 * p + g;
+                sts128(gran(base + OFF_SB + (G >> 3) * kSbCh, n, G & 7),
+                       pack_bf16x2(__uint_as_float(sr[8 * g]), __uint_as_float(sr[8 * g + 1])),
+                       pack_bf16x2(__uint_as_float(sr[8 * g + 2]), __uint_as_float(sr[8 * g + 3])),
+                       pack_bf16x2(__uint_as_float(sr[8 * g + 4]), __uint_as_float(sr[8 * g + 5])),
+                       pack_bf16x2(__uint_as_float(sr[8 * g + 6]), __uint_as_float(sr[8 * g + 7])));
+              }
+            }
           }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_SB));
+      }
+      if (i + 1 < nc) {
+        // the other V1 buffer was last read by chunk i-1's products (done: B_SFULL above)
+        put_v(i + 1, vr);
+        // phi(Q) of chunk i+1 once chunk i's products are done with the operand
+        if (!(ok = bl_warp_wait(bar(B_O1), i & 1, ctl))) break;
+        put_q(qr);
+        load_qv(i + 2, qr, vr);
       }
     }
     // final state, in the layout [1, linear, products] x (64 values | z)
@@ -372,25 +457,21 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
           a.zsum[sb + f] = 0.f;
         }
       } else if (bl_warp_wait(bar(B_SFULL), (nc - 1) & 1, ctl)) {
-        __syncwarp();
         tc_fence_after();
-#pragma unroll 1
-        for (int j = 0; j < 3; ++j) {
-          if (j == 2 && w > 0) break;
-          const int f = 128 * j + 32 * w + lane;
-          uint32_t sr[96];
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j, sr);
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j + 32, sr + 32);
-          tmem_ld32_wait(tmem + lane_t + T_S + 80 * j + 64, sr + 64);
-          if (f < kF) {
-            const long long fa = sb + abi_feature(f);
-            float4* dst = reinterpret_cast<float4*>(a.state + fa * kDV);
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              dst[c] = make_float4(__uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]),
-                                   __uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]));
-            a.zsum[fa] = __uint_as_float(sr[64]);
-          }
+        if (w < 3) {
+          const int n = 32 * w + lane;
+          float* st = a.state + sb * kDV;
+          float* zs = a.zsum + sb;
+          uint32_t sr[32];
+#define SWA_BL_STATE_PIECE(P)                                                               \
+  tmem_ld32_wait(tmem + lane_t + T_ST + 32 * (P), sr);                                      \
+  if (n <= kDV) store_state_piece<P>(sr, n, st, zs, std::make_integer_sequence<int, 32>{});
+          SWA_BL_STATE_PIECE(0)
+          SWA_BL_STATE_PIECE(1)
+          SWA_BL_STATE_PIECE(2)
+          SWA_BL_STATE_PIECE(3)
+          SWA_BL_STATE_PIECE(4)
+#undef SWA_BL_STATE_PIECE
         }
       }
     }
@@ -399,38 +480,37 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
     if (lane == 0 && (a.debug_flags & 1) == 0) {
       bool ok = true;
       for (int i = 0; i < nc && ok; ++i) {
+        const int ob = i & 1;
         if (!(ok = bl_wait(bar(B_PHIQ), i & 1, ctl))) break;
-        if (!(ok = bl_wait(bar(B_V1), i & 1, ctl))) break;
-        if (i > 0) {
-          if (!(ok = bl_wait(bar(B_SB), (i - 1) & 1, ctl))) break;
-          if (!(ok = bl_wait(bar(B_OFREE), (i - 1) & 1, ctl))) break;
-        }
+        if (!(ok = bl_wait(bar(B_PHIK), i & 1, ctl))) break;
         tc_fence_after();
-        // X = phi_lin(Q) phi_lin(K)^T: features 256 .. 271 of phi(Q), columns 0 .. 15 of phi_lin(K)
-        umma_ss<false>(tmem + T_X, bl_kdesc(base + OFF_PHI, kCh, 16), bl_kdesc(base + OFF_KLIN, kCh, 0), IDESC_X, 0u);
+        // X = phi_lin(Q) phi_lin(K)^T: the first 16 feature columns of both operands
+        umma_ss<false>(tmem + T_X, bl_kdesc(base + OFF_PHIQ, kCh, 0), bl_kdesc(base + OFF_PHIK, kCh, 0), IDESC_X, 0u);
         tc_commit(bar(B_X));
         if (i > 0) {
+          if (!(ok = bl_wait(bar(B_SB), (i - 1) & 1, ctl))) break;
+          if (i > 1 && !(ok = bl_wait(bar(B_OFREE + ob), ((i - 2) >> 1) & 1, ctl))) break;
+          tc_fence_after();
 #pragma unroll 1
           for (int kk = 0; kk < kQSteps; ++kk)
-            umma_ss<false>(tmem + T_O, bl_kdesc(base + OFF_PHI, kCh, kk), bl_kdesc(base + OFF_SB, kSbCh, kk),
+            umma_ss<false>(tmem + T_O + 80 * ob, bl_kdesc(base + OFF_PHIQ, kCh, kk), bl_kdesc(base + OFF_SB, kSbCh, kk),
                            IDESC_QS, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(B_O1));
+        const uint32_t v1 = base + OFF_V1 + ob * 2 * kCh;
+        if (!(ok = bl_wait(bar(B_V1 + ob), (i >> 1) & 1, ctl))) break;
         if (!(ok = bl_wait(bar(B_P), i & 1, ctl))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          umma_ts<false>(tmem + T_O, tmem + T_X + kk * 8, bl_mndesc(base + OFF_V1, kCh, kk), IDESC_PV,
+          umma_ts<false>(tmem + T_O + 80 * ob, tmem + T_X + kk * 8, bl_mndesc(v1, kCh, kk), IDESC_PV,
                          (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_OFULL));
-        if (!(ok = bl_wait(bar(B_PHIK), i & 1, ctl))) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int j = 0; j < 3; ++j)
+        tc_commit(bar(B_OFULL + ob));
+        // S^T += V1^T phi(K): A = V1 read MN-major (M = value columns), B = phi(K) MN-major (N = features)
 #pragma unroll
-          for (int kk = 0; kk < kChunk / 16; ++kk)
-            umma_ss<false>(tmem + T_S + 80 * j, bl_mndesc(base + OFF_PHI + 2 * j * kCh, kCh, kk),
-                           bl_mndesc(base + OFF_V1, kCh, kk), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          umma_ss<false>(tmem + T_ST, bl_mndesc(v1, kCh, kk), bl_mndesc(base + OFF_PHIK, kCh, kk), IDESC_KV,
+                         (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_SFULL));
       }
       // let every issued MMA finish before the tensor memory is freed
