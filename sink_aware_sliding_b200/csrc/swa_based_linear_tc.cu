@@ -25,12 +25,14 @@
 // phi(Q) and phi(K) have buffers of their own and V1 and O two each, so the
 // feature rows of the next chunk are written while this chunk's products run.
 //
-// Roles (288 threads):
-//   warps 0-3  token rows of the K side: k loads, phi(K), kappa(X) -> P (bf16,
-//              over X's own tensor-memory columns), the output epilogue;
-//   warps 4-7  token rows of the Q side and state lanes: q and v loads, phi(Q),
-//              V1, S^T -> S_bf16 between chunks, the final state;
-//   warp 8     one thread issues every MMA.
+// Roles (416 threads):
+//   warps 0-3   token rows of the K side: k loads, phi(K), kappa(X) -> P (bf16,
+//               over X's own tensor-memory columns);
+//   warps 4-7   token rows of the Q side and state lanes: q and v loads, phi(Q),
+//               V1, S^T -> S_bf16 between chunks, the final state;
+//   warps 8-11  the output epilogue out = O[:, :64] / O[:, 64];
+//   warp 12     one thread issues every MMA, per chunk in the order X, phi(Q) S,
+//               the state update, P V1 (so that the state update never waits for P).
 // All waits on mbarriers are bounded; on a time-out the CTA stops, drains its
 // MMAs, frees its tensor memory and records the status.
 #include <cuda_bf16.h>
@@ -55,8 +57,8 @@ constexpr int kFReal = kDK + 1 + kDK * (kDK + 1) / 2;   // 153
 constexpr int kNV = 80;                      // V1 columns: 64 values, the ones column, padding
 constexpr int kQSteps = 10;                  // phi(Q) S_bf16 over features 0 .. 159 (K steps of 16)
 constexpr int kGranules = 20;                // 16-byte granules of a feature row written per chunk (0 .. 159)
-constexpr int kThreads = 288;
-constexpr int kMmaWarp = 8;
+constexpr int kThreads = 416;
+constexpr int kMmaWarp = 12;
 constexpr uint32_t kCh = kChunk * 128;       // one 64-column chunk of a 128-row operand: 16 KB
 constexpr uint32_t kSbCh = kNV * 128;        // one 64-column chunk of S_bf16 (80 rows): 10 KB
 constexpr uint32_t OFF_PHIQ = 0;             // [128 tokens x 192 features], 3 chunks
@@ -121,6 +123,30 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t a) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
+// 64 or 96 consecutive columns of this warp's 32 lanes, then one wait::ld (one asm block,
+// so that no register is read before the data has arrived).
+__device__ __forceinline__ void ld64_wait(uint32_t t, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]),"=r"(r[1]),"=r"(r[2]),"=r"(r[3]),"=r"(r[4]),"=r"(r[5]),"=r"(r[6]),"=r"(r[7]),"=r"(r[8]),"=r"(r[9]),"=r"(r[10]),"=r"(r[11]),"=r"(r[12]),"=r"(r[13]),"=r"(r[14]),"=r"(r[15]),"=r"(r[16]),"=r"(r[17]),"=r"(r[18]),"=r"(r[19]),"=r"(r[20]),"=r"(r[21]),"=r"(r[22]),"=r"(r[23]),"=r"(r[24]),"=r"(r[25]),"=r"(r[26]),"=r"(r[27]),"=r"(r[28]),"=r"(r[29]),"=r"(r[30]),"=r"(r[31]),
+        "=r"(r[32]),"=r"(r[33]),"=r"(r[34]),"=r"(r[35]),"=r"(r[36]),"=r"(r[37]),"=r"(r[38]),"=r"(r[39]),"=r"(r[40]),"=r"(r[41]),"=r"(r[42]),"=r"(r[43]),"=r"(r[44]),"=r"(r[45]),"=r"(r[46]),"=r"(r[47]),"=r"(r[48]),"=r"(r[49]),"=r"(r[50]),"=r"(r[51]),"=r"(r[52]),"=r"(r[53]),"=r"(r[54]),"=r"(r[55]),"=r"(r[56]),"=r"(r[57]),"=r"(r[58]),"=r"(r[59]),"=r"(r[60]),"=r"(r[61]),"=r"(r[62]),"=r"(r[63])
+      : "r"(t), "r"(t + 32)
+      : "memory");
+}
+__device__ __forceinline__ void ld96_wait(uint32_t t, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%96];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%97];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%98];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]),"=r"(r[1]),"=r"(r[2]),"=r"(r[3]),"=r"(r[4]),"=r"(r[5]),"=r"(r[6]),"=r"(r[7]),"=r"(r[8]),"=r"(r[9]),"=r"(r[10]),"=r"(r[11]),"=r"(r[12]),"=r"(r[13]),"=r"(r[14]),"=r"(r[15]),"=r"(r[16]),"=r"(r[17]),"=r"(r[18]),"=r"(r[19]),"=r"(r[20]),"=r"(r[21]),"=r"(r[22]),"=r"(r[23]),"=r"(r[24]),"=r"(r[25]),"=r"(r[26]),"=r"(r[27]),"=r"(r[28]),"=r"(r[29]),"=r"(r[30]),"=r"(r[31]),
+        "=r"(r[32]),"=r"(r[33]),"=r"(r[34]),"=r"(r[35]),"=r"(r[36]),"=r"(r[37]),"=r"(r[38]),"=r"(r[39]),"=r"(r[40]),"=r"(r[41]),"=r"(r[42]),"=r"(r[43]),"=r"(r[44]),"=r"(r[45]),"=r"(r[46]),"=r"(r[47]),"=r"(r[48]),"=r"(r[49]),"=r"(r[50]),"=r"(r[51]),"=r"(r[52]),"=r"(r[53]),"=r"(r[54]),"=r"(r[55]),"=r"(r[56]),"=r"(r[57]),"=r"(r[58]),"=r"(r[59]),"=r"(r[60]),"=r"(r[61]),"=r"(r[62]),"=r"(r[63]),
+        "=r"(r[64]),"=r"(r[65]),"=r"(r[66]),"=r"(r[67]),"=r"(r[68]),"=r"(r[69]),"=r"(r[70]),"=r"(r[71]),"=r"(r[72]),"=r"(r[73]),"=r"(r[74]),"=r"(r[75]),"=r"(r[76]),"=r"(r[77]),"=r"(r[78]),"=r"(r[79]),"=r"(r[80]),"=r"(r[81]),"=r"(r[82]),"=r"(r[83]),"=r"(r[84]),"=r"(r[85]),"=r"(r[86]),"=r"(r[87]),"=r"(r[88]),"=r"(r[89]),"=r"(r[90]),"=r"(r[91]),"=r"(r[92]),"=r"(r[93]),"=r"(r[94]),"=r"(r[95])
+      : "r"(t), "r"(t + 32), "r"(t + 64)
+      : "memory");
+}
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
@@ -151,43 +177,6 @@ __device__ __forceinline__ bool bl_warp_wait(uint32_t bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-// Internal feature f (compile-time) of u.
-template <int F>
-__device__ __forceinline__ float feat(const float* u, float rs, float c2, float s) {
-  using namespace bl;
-  if constexpr (F < kDK) {
-    return rs * u[F];
-  } else if constexpr (F == kDK) {
-    return 1.0f;
-  } else if constexpr (F < kFReal) {
-    constexpr int a = pair_a(F - kDK - 1), b = pair_b(F - kDK - 1);
-    return (a == b ? c2 : s) * u[a] * u[b];
-  } else {
-    return 0.0f;
-  }
-}
-template <int G>
-__device__ __forceinline__ void write_granule(uint32_t phi, int t, const float* u, float rs, float c2, float s,
-                                              float keep) {
-  constexpr int f = 8 * G;
-  sts128(gran(phi + (G >> 3) * bl::kCh, t, G & 7),
-         pack_bf16x2(keep * feat<f>(u, rs, c2, s), keep * feat<f + 1>(u, rs, c2, s)),
-         pack_bf16x2(keep * feat<f + 2>(u, rs, c2, s), keep * feat<f + 3>(u, rs, c2, s)),
-         pack_bf16x2(keep * feat<f + 4>(u, rs, c2, s), keep * feat<f + 5>(u, rs, c2, s)),
-         pack_bf16x2(keep * feat<f + 6>(u, rs, c2, s), keep * feat<f + 7>(u, rs, c2, s)));
-}
-template <int... G>
-__device__ __forceinline__ void write_granules(uint32_t phi, int t, const float* u, float rs, float c2, float s,
-                                               float keep, std::integer_sequence<int, G...>) {
-  (write_granule<G>(phi, t, u, rs, c2, s, keep), ...);
-}
-// Row t of phi(u) (internal order, features 0 .. 159) into a K-major feature operand;
-// keep = 0 writes a zero row (tokens past the end of the sequence).
-__device__ __forceinline__ void write_phi_row(uint32_t phi, int t, const float* u, float rs, float c2, float s,
-                                              bool keep) {
-  write_granules(phi, t, u, rs, c2, s, keep ? 1.0f : 0.0f, std::make_integer_sequence<int, bl::kGranules>{});
-}
-
 __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, float* u) {
   const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
@@ -195,6 +184,56 @@ __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, float
     u[2 * i] = bf_lo(w[i]);
     u[2 * i + 1] = bf_hi(w[i]);
   }
+}
+
+// The vectors a feature row is formed from: u, sqrt(scale) u, scale u and
+// scale/sqrt(2) u, and the constant feature (0 for a row past the sequence's end,
+// whose u is zero as well).
+struct FeatIn {
+  float u[bl::kDK], ru[bl::kDK], su[bl::kDK], cu[bl::kDK];
+  float one;
+};
+// Internal feature F (compile-time).
+template <int F>
+__device__ __forceinline__ float feat(const FeatIn& x) {
+  using namespace bl;
+  if constexpr (F < kDK) {
+    return x.ru[F];
+  } else if constexpr (F == kDK) {
+    return x.one;
+  } else if constexpr (F < kFReal) {
+    constexpr int a = pair_a(F - kDK - 1), b = pair_b(F - kDK - 1);
+    return (a == b ? x.cu[a] : x.su[a]) * x.u[b];
+  } else {
+    return 0.0f;
+  }
+}
+template <int G>
+__device__ __forceinline__ void write_granule(uint32_t phi, int t, const FeatIn& x) {
+  constexpr int f = 8 * G;
+  sts128(gran(phi + (G >> 3) * bl::kCh, t, G & 7), pack_bf16x2(feat<f>(x), feat<f + 1>(x)),
+         pack_bf16x2(feat<f + 2>(x), feat<f + 3>(x)), pack_bf16x2(feat<f + 4>(x), feat<f + 5>(x)),
+         pack_bf16x2(feat<f + 6>(x), feat<f + 7>(x)));
+}
+template <int... G>
+__device__ __forceinline__ void write_granules(uint32_t phi, int t, const FeatIn& x, std::integer_sequence<int, G...>) {
+  (write_granule<G>(phi, t, x), ...);
+}
+// Row t of phi(u) (internal order, features 0 .. 159) into a K-major feature operand
+// from the bf16 row (two 16-byte words); keep = false writes a zero row.
+__device__ __forceinline__ void write_phi_row(uint32_t phi, int t, const uint4& lo, const uint4& hi, float rs,
+                                              float c2, float s, bool keep) {
+  FeatIn x;
+  unpack16(lo, hi, x.u);
+#pragma unroll
+  for (int e = 0; e < bl::kDK; ++e) {
+    x.u[e] = keep ? x.u[e] : 0.f;
+    x.ru[e] = rs * x.u[e];
+    x.su[e] = s * x.u[e];
+    x.cu[e] = c2 * x.u[e];
+  }
+  x.one = keep ? 1.0f : 0.0f;
+  write_granules(phi, t, x, std::make_integer_sequence<int, bl::kGranules>{});
 }
 
 // Internal feature F of one state lane (value column n < 64, or z for n = 64) into the
@@ -229,7 +268,7 @@ __device__ __forceinline__ void store_state_piece(const uint32_t* sr, int n, flo
   (store_state_feature<32 * P + E>(__uint_as_float(sr[E]), n, st, zs), ...);
 }
 
-__global__ void __launch_bounds__(bl::kThreads, 1)
+__global__ void __maxnreg__(152)
     swa_based_linear_tc_kernel(const __grid_constant__ BasedLinearArgs a) {
   using namespace bl;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -301,11 +340,7 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       load_k(i + 1, nxt);
       // phi(K) once the previous chunk's products are done with the operand
       if (i > 0 && !(ok = bl_warp_wait(bar(B_SFULL), (i - 1) & 1, ctl))) break;
-      {
-        float u[16];
-        unpack16(cur[0], cur[1], u);
-        write_phi_row(base + OFF_PHIK, t, u, rs, c2, sc, t < n);
-      }
+      write_phi_row(base + OFF_PHIK, t, cur[0], cur[1], rs, c2, sc, t < n);
       fence_proxy_async_smem();
       mbar_arrive(bar(B_PHIK));
       // kappa(X) with the causal mask -> P (bf16 pairs over X's first 64 columns)
@@ -314,8 +349,7 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t xr[64], pr[32];
-        tmem_ld32_wait(tmem + lane_t + T_X + 64 * half, xr);
-        tmem_ld32_wait(tmem + lane_t + T_X + 64 * half + 32, xr + 32);
+        ld64_wait(tmem + lane_t + T_X + 64 * half, xr);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int s0 = 64 * half + 2 * j;
@@ -329,37 +363,6 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P));
-      // epilogue: out = O[:, :64] / O[:, 64]
-      const int ob = i & 1;
-      if (!(ok = bl_warp_wait(bar(B_OFULL + ob), (i >> 1) & 1, ctl))) break;
-      tc_fence_after();
-      uint32_t orr[96];
-      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob, orr);
-      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob + 32, orr + 32);
-      tmem_ld32_wait(tmem + lane_t + T_O + 80 * ob + 64, orr + 64);
-      tc_fence_before();
-      mbar_arrive(bar(B_OFREE + ob));
-      if (t < n) {
-        const float inv = 1.0f / __uint_as_float(orr[64]);
-        const long long row = (static_cast<long long>(b) * a.L + i * kChunk + t) * a.H + h;
-        if (a.out_f32) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * kDV);
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            o[c] = make_float4(__uint_as_float(orr[4 * c]) * inv, __uint_as_float(orr[4 * c + 1]) * inv,
-                               __uint_as_float(orr[4 * c + 2]) * inv, __uint_as_float(orr[4 * c + 3]) * inv);
-        } else {
-          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * kDV);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t* w = orr + 8 * c;
-            o[c] = make_uint4(pack_bf16x2(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv),
-                              pack_bf16x2(__uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv),
-                              pack_bf16x2(__uint_as_float(w[4]) * inv, __uint_as_float(w[5]) * inv),
-                              pack_bf16x2(__uint_as_float(w[6]) * inv, __uint_as_float(w[7]) * inv));
-          }
-        }
-      }
       cur[0] = nxt[0];
       cur[1] = nxt[1];
     }
@@ -395,9 +398,7 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       mbar_arrive(bar(B_V1 + (c & 1)));
     };
     auto put_q = [&](const uint4* qr) {
-      float u[16];
-      unpack16(qr[0], qr[1], u);
-      write_phi_row(base + OFF_PHIQ, r, u, rs, c2, sc, true);
+      write_phi_row(base + OFF_PHIQ, r, qr[0], qr[1], rs, c2, sc, true);
       fence_proxy_async_smem();
       mbar_arrive(bar(B_PHIQ));
     };
@@ -417,12 +418,13 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         if (w < 3) {
           const int n = 32 * w + lane;
 #pragma unroll
-          for (int p = 0; p < 5; ++p) {
-            uint32_t sr[32];
-            tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
+          for (int p = 0; p < 5; p += 2) {                 // columns 64 p' .. : 64, 64, 32
+            uint32_t sr[64];
+            if (p < 4) ld64_wait(tmem + lane_t + T_ST + 32 * p, sr);
+            else tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
             if (n < kNV) {
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
+              for (int g = 0; g < (p < 4 ? 8 : 4); ++g) {
                 const int G = 4 * p + g;
                 sts128(gran(base + OFF_SB + (G >> 3) * kSbCh, n, G & 7),
                        pack_bf16x2(__uint_as_float(sr[8 * g]), __uint_as_float(sr[8 * g + 1])),
@@ -438,7 +440,9 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         mbar_arrive(bar(B_SB));
       }
       if (i + 1 < nc) {
-        // the other V1 buffer was last read by chunk i-1's products (done: B_SFULL above)
+        // the other V1 buffer was last read by chunk i-1's state update (done: B_SFULL
+        // above) and its P V1, issued after it
+        if (i > 0 && !(ok = bl_warp_wait(bar(B_OFULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, ctl))) break;
         put_v(i + 1, vr);
         // phi(Q) of chunk i+1 once chunk i's products are done with the operand
         if (!(ok = bl_warp_wait(bar(B_O1), i & 1, ctl))) break;
@@ -475,6 +479,41 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         }
       }
     }
+  } else if (warp < 12) {
+    // ---------------------------------------------------------------- output epilogue
+    const int t = tid - 256;                             // row of the chunk = tensor-memory lane
+    const uint32_t lane_t = static_cast<uint32_t>((warp - 8) * 32) << 16;
+    for (int i = 0; i < nc; ++i) {
+      const int n = min(kChunk, a.L - i * kChunk);
+      const int ob = i & 1;
+      if (!bl_warp_wait(bar(B_OFULL + ob), (i >> 1) & 1, ctl)) break;
+      tc_fence_after();
+      uint32_t orr[96];
+      ld96_wait(tmem + lane_t + T_O + 80 * ob, orr);
+      tc_fence_before();
+      mbar_arrive(bar(B_OFREE + ob));
+      if (t < n) {
+        const float inv = 1.0f / __uint_as_float(orr[64]);
+        const long long row = (static_cast<long long>(b) * a.L + i * kChunk + t) * a.H + h;
+        if (a.out_f32) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * kDV);
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            o[c] = make_float4(__uint_as_float(orr[4 * c]) * inv, __uint_as_float(orr[4 * c + 1]) * inv,
+                               __uint_as_float(orr[4 * c + 2]) * inv, __uint_as_float(orr[4 * c + 3]) * inv);
+        } else {
+          uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * kDV);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* w = orr + 8 * c;
+            o[c] = make_uint4(pack_bf16x2(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv),
+                              pack_bf16x2(__uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv),
+                              pack_bf16x2(__uint_as_float(w[4]) * inv, __uint_as_float(w[5]) * inv),
+                              pack_bf16x2(__uint_as_float(w[6]) * inv, __uint_as_float(w[7]) * inv));
+          }
+        }
+      }
+    }
   } else {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && (a.debug_flags & 1) == 0) {
@@ -483,6 +522,8 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         const int ob = i & 1;
         if (!(ok = bl_wait(bar(B_PHIQ), i & 1, ctl))) break;
         if (!(ok = bl_wait(bar(B_PHIK), i & 1, ctl))) break;
+        // X overwrites P: chunk i-1's P V1 must be done
+        if (i > 0 && !(ok = bl_wait(bar(B_OFULL + (ob ^ 1)), ((i - 1) >> 1) & 1, ctl))) break;
         tc_fence_after();
         // X = phi_lin(Q) phi_lin(K)^T: the first 16 feature columns of both operands
         umma_ss<false>(tmem + T_X, bl_kdesc(base + OFF_PHIQ, kCh, 0), bl_kdesc(base + OFF_PHIK, kCh, 0), IDESC_X, 0u);
@@ -499,6 +540,13 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         tc_commit(bar(B_O1));
         const uint32_t v1 = base + OFF_V1 + ob * 2 * kCh;
         if (!(ok = bl_wait(bar(B_V1 + ob), (i >> 1) & 1, ctl))) break;
+        tc_fence_after();
+        // S^T += V1^T phi(K): A = V1 read MN-major (M = value columns), B = phi(K) MN-major (N = features)
+#pragma unroll
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          umma_ss<false>(tmem + T_ST, bl_mndesc(v1, kCh, kk), bl_mndesc(base + OFF_PHIK, kCh, kk), IDESC_KV,
+                         (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(B_SFULL));
         if (!(ok = bl_wait(bar(B_P), i & 1, ctl))) break;
         tc_fence_after();
 #pragma unroll
@@ -506,12 +554,6 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
           umma_ts<false>(tmem + T_O + 80 * ob, tmem + T_X + kk * 8, bl_mndesc(v1, kCh, kk), IDESC_PV,
                          (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_OFULL + ob));
-        // S^T += V1^T phi(K): A = V1 read MN-major (M = value columns), B = phi(K) MN-major (N = features)
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          umma_ss<false>(tmem + T_ST, bl_mndesc(v1, kCh, kk), bl_mndesc(base + OFF_PHIK, kCh, kk), IDESC_KV,
-                         (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_SFULL));
       }
       // let every issued MMA finish before the tensor memory is freed
       tc_commit(bar(B_DRAIN));
