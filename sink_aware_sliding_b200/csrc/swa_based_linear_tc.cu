@@ -268,7 +268,9 @@ __device__ __forceinline__ void store_state_piece(const uint32_t* sr, int n, flo
   (store_state_feature<32 * P + E>(__uint_as_float(sr[E]), n, st, zs), ...);
 }
 
-__global__ void __maxnreg__(152)
+// 13 warps: one of the four SM sub-partitions holds four of them, and its 16K
+// registers cap every thread at 128 (ptxas applies the cap from these bounds).
+__global__ void __launch_bounds__(bl::kThreads, 1)
     swa_based_linear_tc_kernel(const __grid_constant__ BasedLinearArgs a) {
   using namespace bl;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
