@@ -419,14 +419,13 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         tc_fence_after();
         if (w < 3) {
           const int n = 32 * w + lane;
-#pragma unroll
-          for (int p = 0; p < 5; p += 2) {                 // columns 64 p' .. : 64, 64, 32
-            uint32_t sr[64];
-            if (p < 4) ld64_wait(tmem + lane_t + T_ST + 32 * p, sr);
-            else tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
+#pragma unroll 1
+          for (int p = 0; p < 5; ++p) {
+            uint32_t sr[32];
+            tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
             if (n < kNV) {
 #pragma unroll
-              for (int g = 0; g < (p < 4 ? 8 : 4); ++g) {
+              for (int g = 0; g < 4; ++g) {
                 const int G = 4 * p + g;
                 sts128(gran(base + OFF_SB + (G >> 3) * kSbCh, n, G & 7),
                        pack_bf16x2(__uint_as_float(sr[8 * g]), __uint_as_float(sr[8 * g + 1])),
