@@ -65,7 +65,9 @@ constexpr uint32_t OFF_PHIQ = 0;             // [128 tokens x 192 features], 3 c
 constexpr uint32_t OFF_PHIK = 3 * kCh;
 constexpr uint32_t OFF_V1 = 6 * kCh;         // two buffers of [values chunk | ones chunk]
 constexpr uint32_t OFF_SB = 10 * kCh;        // S_bf16 [80 value columns x 192 features], 3 chunks
-constexpr uint32_t OFF_BAR = OFF_SB + 3 * kSbCh;
+constexpr uint32_t OFF_QST = OFF_SB + 3 * kSbCh;   // q rows of two chunks (32 bytes a row)
+constexpr uint32_t OFF_KST = OFF_QST + 2 * kChunk * 32;  // k rows of two chunks
+constexpr uint32_t OFF_BAR = OFF_KST + 2 * kChunk * 32;
 enum {
   B_PHIQ, B_PHIK, B_V1, B_V1b, B_X, B_O1, B_P, B_OFULL, B_OFULLb, B_OFREE, B_OFREEb, B_SFULL, B_SB, B_DRAIN,
   kNumBars
@@ -149,6 +151,23 @@ __device__ __forceinline__ void ld96_wait(uint32_t t, uint32_t* r) {
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 16-byte asynchronous copy global -> shared (zero-filled when src_bytes = 0); the
+// copies are tracked by commit groups, not by the thread's registers, so a later
+// barrier wait does not wait for them.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
 
 struct BlCtl {
   volatile int* abort_flag;
@@ -324,27 +343,31 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
     const int t = tid;                                   // row of the chunk = tensor-memory lane
     const uint32_t lane_t = static_cast<uint32_t>(warp * 32) << 16;
     const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
-    auto load_k = [&](int i, uint4* r) {
-      const int tok = i * kChunk + t;
-      if (i < nc && tok < a.L) {
-        const uint4* pk = reinterpret_cast<const uint4*>(kg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDK);
-        r[0] = __ldg(pk);
-        r[1] = __ldg(pk + 1);
-      } else {
-        r[0] = r[1] = make_uint4(0, 0, 0, 0);
-      }
+    // k row t of chunk c -> staging buffer c & 1 (a commit group of its own)
+    auto copy_k = [&](int c) {
+      const int tok = c * kChunk + t;
+      const bool in = c < nc && tok < a.L;
+      const __nv_bfloat16* src = in ? kg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDK : kg;
+      const uint32_t dst = base + OFF_KST + (c & 1) * kChunk * 32 + t * 32;
+      cp_async16(dst, src, in ? 16u : 0u);
+      cp_async16(dst + 16, src + 8, in ? 16u : 0u);
+      cp_async_commit();
     };
-    uint4 cur[2], nxt[2];
-    load_k(0, cur);
+    copy_k(0);
+    copy_k(1);
     bool ok = true;
     for (int i = 0; i < nc && ok; ++i) {
       const int n = min(kChunk, a.L - i * kChunk);
-      load_k(i + 1, nxt);
       // phi(K) once the previous chunk's products are done with the operand
       if (i > 0 && !(ok = bl_warp_wait(bar(B_SFULL), (i - 1) & 1, ctl))) break;
-      write_phi_row(base + OFF_PHIK, t, cur[0], cur[1], rs, c2, sc, t < n);
+      cp_async_wait<1>();                                // k of chunk i (chunk i+1's may be in flight)
+      {
+        const uint32_t src = base + OFF_KST + (i & 1) * kChunk * 32 + t * 32;
+        write_phi_row(base + OFF_PHIK, t, lds128(src), lds128(src + 16), rs, c2, sc, t < n);
+      }
       fence_proxy_async_smem();
       mbar_arrive(bar(B_PHIK));
+      copy_k(i + 2);                                     // into the buffer just read
       // kappa(X) with the causal mask -> P (bf16 pairs over X's first 64 columns)
       if (!(ok = bl_warp_wait(bar(B_X), i & 1, ctl))) break;
       tc_fence_after();
@@ -365,9 +388,8 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P));
-      cur[0] = nxt[0];
-      cur[1] = nxt[1];
     }
+    cp_async_wait<0>();
   } else if (warp < 8) {
     // ---------------------------------------------------------------- Q-side token rows, state lanes
     const int r = tid - 128;                             // token row (phi(Q), V1) and state lane
@@ -375,42 +397,45 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
     const uint32_t lane_t = static_cast<uint32_t>(w * 32) << 16;
     const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
     const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
-    auto load_qv = [&](int i, uint4* qr, uint4* vr) {
-      const int tok = i * kChunk + r;
-      if (i < nc && tok < a.L) {
-        const long long row = (static_cast<long long>(b) * a.L + tok) * a.H + h;
-        const uint4* pq = reinterpret_cast<const uint4*>(qg + row * kDK);
-        const uint4* pv = reinterpret_cast<const uint4*>(vg + row * kDV);
-        qr[0] = __ldg(pq);
-        qr[1] = __ldg(pq + 1);
-#pragma unroll
-        for (int g = 0; g < 8; ++g) vr[g] = __ldg(pv + g);
-      } else {
-        qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int g = 0; g < 8; ++g) vr[g] = make_uint4(0, 0, 0, 0);
-      }
-    };
-    // chunk c's values into V1 buffer c & 1 and phi(Q) of chunk c
-    auto put_v = [&](int c, const uint4* vr) {
+    // Asynchronous copies of chunk c: its v rows into V1 buffer c & 1 (16-byte granules,
+    // swizzled as the MMA reads them) and its q rows into staging buffer c & 1.  Each
+    // call is one commit group.
+    auto copy_v = [&](int c) {
+      const int tok = c * kChunk + r;
+      const bool in = c < nc && tok < a.L;
+      const __nv_bfloat16* src = in ? vg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDV : vg;
       const uint32_t vb = base + OFF_V1 + (c & 1) * 2 * kCh;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) sts128(gran(vb, r, g), vr[g].x, vr[g].y, vr[g].z, vr[g].w);
+      for (int g = 0; g < 8; ++g) cp_async16(gran(vb, r, g), src + 8 * g, in ? 16u : 0u);
+      cp_async_commit();
+    };
+    auto copy_q = [&](int c) {
+      const int tok = c * kChunk + r;
+      const bool in = c < nc && tok < a.L;
+      const __nv_bfloat16* src = in ? qg + ((static_cast<long long>(b) * a.L + tok) * a.H + h) * kDK : qg;
+      const uint32_t dst = base + OFF_QST + (c & 1) * kChunk * 32 + r * 32;
+      cp_async16(dst, src, in ? 16u : 0u);
+      cp_async16(dst + 16, src + 8, in ? 16u : 0u);
+      cp_async_commit();
+    };
+    auto v_ready = [&](int c) {                          // after its copies have landed
       fence_proxy_async_smem();
       mbar_arrive(bar(B_V1 + (c & 1)));
     };
-    auto put_q = [&](const uint4* qr) {
-      write_phi_row(base + OFF_PHIQ, r, qr[0], qr[1], rs, c2, sc, true);
+    auto put_q = [&](int c) {                            // after its copies have landed
+      const uint32_t src = base + OFF_QST + (c & 1) * kChunk * 32 + r * 32;
+      write_phi_row(base + OFF_PHIQ, r, lds128(src), lds128(src + 16), rs, c2, sc, true);
       fence_proxy_async_smem();
       mbar_arrive(bar(B_PHIQ));
     };
-    uint4 qr[2], vr[8];
     bool ok = true;
     if (nc > 0) {
-      load_qv(0, qr, vr);
-      put_v(0, vr);
-      put_q(qr);
-      load_qv(1, qr, vr);
+      copy_v(0);
+      copy_q(0);
+      cp_async_wait<0>();
+      v_ready(0);
+      put_q(0);
+      copy_q(1);
     }
     for (int i = 0; i < nc && ok; ++i) {
       if (i > 0) {
@@ -440,17 +465,24 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(B_SB));
       }
+      // commit groups in flight: at most [v(i)], [q(i+1)] (issued in the previous round)
+      if (i > 0) {
+        cp_async_wait<1>();                              // v(i) landed
+        v_ready(i);
+      }
       if (i + 1 < nc) {
         // the other V1 buffer was last read by chunk i-1's state update (done: B_SFULL
         // above) and its P V1, issued after it
         if (i > 0 && !(ok = bl_warp_wait(bar(B_OFULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, ctl))) break;
-        put_v(i + 1, vr);
+        copy_v(i + 1);
         // phi(Q) of chunk i+1 once chunk i's products are done with the operand
         if (!(ok = bl_warp_wait(bar(B_O1), i & 1, ctl))) break;
-        put_q(qr);
-        load_qv(i + 2, qr, vr);
+        cp_async_wait<1>();                              // q(i+1) landed (v(i+1) may be in flight)
+        put_q(i + 1);
+        copy_q(i + 2);
       }
     }
+    cp_async_wait<0>();
     // final state, in the layout [1, linear, products] x (64 values | z)
     if (ok && a.state != nullptr) {
       const long long sb = static_cast<long long>(bh) * kF;
