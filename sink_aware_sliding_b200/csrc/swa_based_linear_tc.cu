@@ -30,8 +30,8 @@
 //               over X's own tensor-memory columns);
 //   warps 4-7   token rows of the Q side and state lanes: q and v loads, phi(Q),
 //               V1, S^T -> S_bf16 between chunks, the final state;
-//   warps 8-11  the output epilogue out = O[:, :64] / O[:, 64];
-//   warp 12     one thread issues every MMA, per chunk in the order X, phi(Q) S,
+//   warps 8-11  part of S^T -> S_bf16, the output epilogue out = O[:, :64] / O[:, 64];
+//   warp 12     one thread issues every MMA, per chunk in the order phi(Q) S, X,
 //               the state update, P V1 (so that the state update never waits for P).
 // All waits on mbarriers are bounded; on a time-out the CTA stops, drains its
 // MMAs, frees its tensor memory and records the status.
@@ -287,6 +287,27 @@ __device__ __forceinline__ void store_state_piece(const uint32_t* sr, int n, flo
   (store_state_feature<32 * P + E>(__uint_as_float(sr[E]), n, st, zs), ...);
 }
 
+// S^T columns 32 p0 .. 32 p1 - 1 (features) of this warp's lanes -> rows of S_bf16
+// (lane n = value column; lanes 80 and up hold nothing).  Warp-collective.
+__device__ __forceinline__ void convert_state(uint32_t tmem_lane, uint32_t sb, int n, int p0, int p1) {
+#pragma unroll 1
+  for (int p = p0; p < p1; ++p) {
+    uint32_t sr[32];
+    tmem_ld32_wait(tmem_lane + bl::T_ST + 32 * p, sr);
+    if (n < bl::kNV) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int G = 4 * p + g;
+        sts128(gran(sb + (G >> 3) * bl::kSbCh, n, G & 7),
+               pack_bf16x2(__uint_as_float(sr[8 * g]), __uint_as_float(sr[8 * g + 1])),
+               pack_bf16x2(__uint_as_float(sr[8 * g + 2]), __uint_as_float(sr[8 * g + 3])),
+               pack_bf16x2(__uint_as_float(sr[8 * g + 4]), __uint_as_float(sr[8 * g + 5])),
+               pack_bf16x2(__uint_as_float(sr[8 * g + 6]), __uint_as_float(sr[8 * g + 7])));
+      }
+    }
+  }
+}
+
 // 13 warps: one of the four SM sub-partitions holds four of them, and its 16K
 // registers cap every thread at 128 (ptxas applies the cap from these bounds).
 __global__ void __launch_bounds__(bl::kThreads, 1)
@@ -322,8 +343,8 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       const bool threads = i == B_PHIQ || i == B_PHIK || i == B_V1 || i == B_V1b || i == B_P || i == B_OFREE ||
-                           i == B_OFREEb || i == B_SB;
-      mbar_init(bar(i), threads ? 128 : 1);
+                           i == B_OFREEb;
+      mbar_init(bar(i), i == B_SB ? 256 : (threads ? 128 : 1));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -442,25 +463,8 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
         // S^T after chunk i-1 -> S_bf16 (row n = value column, K-major over the features)
         if (!(ok = bl_warp_wait(bar(B_SFULL), (i - 1) & 1, ctl))) break;
         tc_fence_after();
-        if (w < 3) {
-          const int n = 32 * w + lane;
-#pragma unroll 1
-          for (int p = 0; p < 5; ++p) {
-            uint32_t sr[32];
-            tmem_ld32_wait(tmem + lane_t + T_ST + 32 * p, sr);
-            if (n < kNV) {
-#pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const int G = 4 * p + g;
-                sts128(gran(base + OFF_SB + (G >> 3) * kSbCh, n, G & 7),
-                       pack_bf16x2(__uint_as_float(sr[8 * g]), __uint_as_float(sr[8 * g + 1])),
-                       pack_bf16x2(__uint_as_float(sr[8 * g + 2]), __uint_as_float(sr[8 * g + 3])),
-                       pack_bf16x2(__uint_as_float(sr[8 * g + 4]), __uint_as_float(sr[8 * g + 5])),
-                       pack_bf16x2(__uint_as_float(sr[8 * g + 6]), __uint_as_float(sr[8 * g + 7])));
-              }
-            }
-          }
-        }
+        // features 0 .. 95 here, 96 .. 159 in the epilogue warps
+        if (w < 3) convert_state(tmem + lane_t, base + OFF_SB, 32 * w + lane, 0, 3);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_SB));
@@ -519,6 +523,16 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
     for (int i = 0; i < nc; ++i) {
       const int n = min(kChunk, a.L - i * kChunk);
       const int ob = i & 1;
+      if (i + 1 < nc) {
+        // features 96 .. 159 of S^T after chunk i -> S_bf16 for chunk i+1 (the rest in
+        // warps 4-6); the state update of chunk i completes before its P V1
+        if (!bl_warp_wait(bar(B_SFULL), i & 1, ctl)) break;
+        tc_fence_after();
+        if (warp < 11) convert_state(tmem + lane_t, base + OFF_SB, t, 3, 5);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_SB));
+      }
       if (!bl_warp_wait(bar(B_OFULL + ob), (i >> 1) & 1, ctl)) break;
       tc_fence_after();
       uint32_t orr[96];
@@ -554,14 +568,8 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       for (int i = 0; i < nc && ok; ++i) {
         const int ob = i & 1;
         if (!(ok = bl_wait(bar(B_PHIQ), i & 1, ctl))) break;
-        if (!(ok = bl_wait(bar(B_PHIK), i & 1, ctl))) break;
-        // X overwrites P: chunk i-1's P V1 must be done
-        if (i > 0 && !(ok = bl_wait(bar(B_OFULL + (ob ^ 1)), ((i - 1) >> 1) & 1, ctl))) break;
-        tc_fence_after();
-        // X = phi_lin(Q) phi_lin(K)^T: the first 16 feature columns of both operands
-        umma_ss<false>(tmem + T_X, bl_kdesc(base + OFF_PHIQ, kCh, 0), bl_kdesc(base + OFF_PHIK, kCh, 0), IDESC_X, 0u);
-        tc_commit(bar(B_X));
         if (i > 0) {
+          // O = phi(Q) S_bf16 needs phi(Q), the converted state and a drained O buffer
           if (!(ok = bl_wait(bar(B_SB), (i - 1) & 1, ctl))) break;
           if (i > 1 && !(ok = bl_wait(bar(B_OFREE + ob), ((i - 2) >> 1) & 1, ctl))) break;
           tc_fence_after();
@@ -570,6 +578,13 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
             umma_ss<false>(tmem + T_O + 80 * ob, bl_kdesc(base + OFF_PHIQ, kCh, kk), bl_kdesc(base + OFF_SB, kSbCh, kk),
                            IDESC_QS, kk > 0 ? 1u : 0u);
         }
+        if (!(ok = bl_wait(bar(B_PHIK), i & 1, ctl))) break;
+        // X overwrites P: chunk i-1's P V1 must be done
+        if (i > 0 && !(ok = bl_wait(bar(B_OFULL + (ob ^ 1)), ((i - 1) >> 1) & 1, ctl))) break;
+        tc_fence_after();
+        // X = phi_lin(Q) phi_lin(K)^T: the first 16 feature columns of both operands
+        umma_ss<false>(tmem + T_X, bl_kdesc(base + OFF_PHIQ, kCh, 0), bl_kdesc(base + OFF_PHIK, kCh, 0), IDESC_X, 0u);
+        tc_commit(bar(B_X));
         tc_commit(bar(B_O1));
         const uint32_t v1 = base + OFF_V1 + ob * 2 * kCh;
         if (!(ok = bl_wait(bar(B_V1 + ob), (i >> 1) & 1, ctl))) break;
