@@ -17,12 +17,9 @@
 // V1 = [V | 1 | 0...] (the values, a column of ones that turns the same products
 // into the normaliser, zero padding) a chunk is
 //   X   = phi_lin(Q) phi_lin(K)^T                  (= scale q.k; K = 16)
-//   O   = phi(Q) S_bf16 + kappa_causal(X) V          (S from the earlier chunks)
+//   O   = phi(Q) S_bf16 + kappa_causal(X) V1        (S from the earlier chunks)
 //   S^T += V1^T phi(K)                              (M = value column, N = 192 features)
-// with kappa(x) = 1 + x + x^2/2 under the causal mask.  The normaliser is column 64
-// of phi(Q) S_bf16 (phi(q).z) plus the row sum of kappa_causal(X), which the kappa
-// warps add up themselves, so that P V reads the values as one whole swizzle atom;
-// out = O[:, :64] / (O[:, 64] + O[:, 65]).
+// with kappa(x) = 1 + x + x^2/2 under the causal mask and out = O[:, :64] / O[:, 64].
 // S is accumulated transposed (tensor-memory lane = value column), so that each
 // lane's row is one row of the K-major bf16 operand of the next chunk's phi(Q) S.
 // phi(Q) and phi(K) have buffers of their own and V1 and O two each, so the
@@ -87,7 +84,7 @@ constexpr uint32_t T_ST = 288;               // S^T: lanes = value columns, 192 
 // instruction descriptors (bf16 x bf16 -> fp32); bit 15 makes A MN-major
 constexpr uint32_t IDESC_X = make_idesc(1, 128, 128, false);
 constexpr uint32_t IDESC_QS = make_idesc(1, 128, kNV, false);
-constexpr uint32_t IDESC_PV = make_idesc(1, 128, kDV, true);   // values only: one whole swizzle atom
+constexpr uint32_t IDESC_PV = make_idesc(1, 128, kNV, true);
 constexpr uint32_t IDESC_KV = make_idesc(1, 128, kFI, true) | (1u << 15);
 constexpr int kStatusTimeout = 4;            // SWA_ERR_DEVICE_TIMEOUT
 
@@ -151,10 +148,6 @@ __device__ __forceinline__ void ld96_wait(uint32_t t, uint32_t* r) {
         "=r"(r[64]),"=r"(r[65]),"=r"(r[66]),"=r"(r[67]),"=r"(r[68]),"=r"(r[69]),"=r"(r[70]),"=r"(r[71]),"=r"(r[72]),"=r"(r[73]),"=r"(r[74]),"=r"(r[75]),"=r"(r[76]),"=r"(r[77]),"=r"(r[78]),"=r"(r[79]),"=r"(r[80]),"=r"(r[81]),"=r"(r[82]),"=r"(r[83]),"=r"(r[84]),"=r"(r[85]),"=r"(r[86]),"=r"(r[87]),"=r"(r[88]),"=r"(r[89]),"=r"(r[90]),"=r"(r[91]),"=r"(r[92]),"=r"(r[93]),"=r"(r[94]),"=r"(r[95])
       : "r"(t), "r"(t + 32), "r"(t + 64)
       : "memory");
-}
-// One 32-bit column of this warp's 32 lanes.
-__device__ __forceinline__ void tmem_st1(uint32_t t, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(t), "r"(v) : "memory");
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -399,10 +392,6 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       // kappa(X) with the causal mask -> P (bf16 pairs over X's first 64 columns)
       if (!(ok = bl_warp_wait(bar(B_X), i & 1, ctl))) break;
       tc_fence_after();
-      // The row sums of the bf16 kappa values (what P V1 would add to the ones column)
-      // go to column 65 of this chunk's O buffer, which phi(Q) S (issued before X, so
-      // already complete) has written; P V1 covers only the 64 value columns.
-      float rsum = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t xr[64], pr[32];
@@ -414,11 +403,9 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
           const float k0 = s0 <= t ? fmaf(x0, fmaf(0.5f, x0, 1.f), 1.f) : 0.f;
           const float k1 = s0 + 1 <= t ? fmaf(x1, fmaf(0.5f, x1, 1.f), 1.f) : 0.f;
           pr[j] = pack_bf16x2(k0, k1);
-          rsum += bf_lo(pr[j]) + bf_hi(pr[j]);
         }
         tmem_st32(tmem + lane_t + T_X + 32 * half, pr);
       }
-      tmem_st1(tmem + lane_t + T_O + 80 * (i & 1) + kDV + 1, __float_as_uint(rsum));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P));
@@ -553,9 +540,7 @@ __global__ void __launch_bounds__(bl::kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_OFREE + ob));
       if (t < n) {
-        // normaliser: phi(q).z of the earlier chunks (column 64; none before chunk 1)
-        // plus the row sum of this chunk's kernel values (column 65)
-        const float inv = 1.0f / ((i > 0 ? __uint_as_float(orr[64]) : 0.f) + __uint_as_float(orr[65]));
+        const float inv = 1.0f / __uint_as_float(orr[64]);
         const long long row = (static_cast<long long>(b) * a.L + i * kChunk + t) * a.H + h;
         if (a.out_f32) {
           float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + row * kDV);
