@@ -295,8 +295,11 @@ unsigned long long swa_set_wait_timeout_ns(unsigned long long ns);
  * no copies, so that its consumers' bounded waits run out; bit 1 makes
  * swa_fwd / swa_fwd_varlen use the one-query-tile kernel even where another
  * kernel applies; bit 2 keeps them off the short-window stream kernel (d = 64,
- * window <= 129, no sinks), so the two-tile kernel runs instead.  0 restores
- * normal operation.  Returns the previous flags.
+ * window <= 129, no sinks), so the two-tile kernel runs instead.  For
+ * swa_based_linear_fwd, bit 0 makes the MMA warp issue nothing (the other warps'
+ * bounded waits run out) and bit 3 runs the fp32 CUDA-core form of the same
+ * chunked step instead of the tensor-core kernel.  0 restores normal operation.
+ * Returns the previous flags.
  */
 int swa_set_debug_flags(int flags);
 
