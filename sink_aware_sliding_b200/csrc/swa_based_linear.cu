@@ -152,13 +152,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // One decode step per (sequence, head): S += phi(k) v^T, z += phi(k), out = phi(q) S / phi(q).z.
 // 256 threads: thread (c4, g) owns columns 4 c4 .. 4 c4 + 3 of S for the features
-// f = g, g + 16, ...; the loads of a thread's rows are issued in batches so that
-// several 16-byte reads are in flight per thread (the step is HBM-bound).
+// f = g, g + 16, ...; its rows are read in two batches of nine 16-byte loads, all
+// in flight at once, and the kernel keeps to 64 registers so that four CTAs share
+// an SM and one CTA's stores overlap another's loads (the step is HBM-bound).
 constexpr int kDecThreads = 256;
 constexpr int kDecGroups = kDecThreads / (kDV / 4);        // 16
 constexpr int kDecRows = (kF + kDecGroups - 1) / kDecGroups;  // 18 rows per group at most
 
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 4)
     swa_based_linear_decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                    const __nv_bfloat16* __restrict__ v, float* __restrict__ state,
                                    float* __restrict__ zsum, void* __restrict__ out, int H, float scale, int out_f32) {
@@ -186,28 +187,32 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   __syncthreads();
   float4* S4 = reinterpret_cast<float4*>(state + bh * kF * kDV) + c4;
-  float4 row[kDecRows];
-#pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    const int f = g + kDecGroups * i;
-    if (f < kF) row[i] = S4[f * (kDV / 4)];
-  }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // two batches of kDecRows / 2 rows: all loads of a batch in flight, then the updates
 #pragma unroll
-  for (int i = 0; i < kDecRows; ++i) {
-    const int f = g + kDecGroups * i;
-    if (f < kF) {
-      const float a = fk[f], b = fq[f];
-      float4 r = row[i];
-      r.x = fmaf(a, vv.x, r.x);
-      r.y = fmaf(a, vv.y, r.y);
-      r.z = fmaf(a, vv.z, r.z);
-      r.w = fmaf(a, vv.w, r.w);
-      S4[f * (kDV / 4)] = r;
-      acc.x = fmaf(b, r.x, acc.x);
-      acc.y = fmaf(b, r.y, acc.y);
-      acc.z = fmaf(b, r.z, acc.z);
-      acc.w = fmaf(b, r.w, acc.w);
+  for (int h0 = 0; h0 < kDecRows; h0 += kDecRows / 2) {
+    float4 row[kDecRows / 2];
+#pragma unroll
+    for (int i = 0; i < kDecRows / 2; ++i) {
+      const int f = g + kDecGroups * (h0 + i);
+      if (f < kF) row[i] = S4[f * (kDV / 4)];
+    }
+#pragma unroll
+    for (int i = 0; i < kDecRows / 2; ++i) {
+      const int f = g + kDecGroups * (h0 + i);
+      if (f < kF) {
+        const float a = fk[f], b = fq[f];
+        float4 r = row[i];
+        r.x = fmaf(a, vv.x, r.x);
+        r.y = fmaf(a, vv.y, r.y);
+        r.z = fmaf(a, vv.z, r.z);
+        r.w = fmaf(a, vv.w, r.w);
+        S4[f * (kDV / 4)] = r;
+        acc.x = fmaf(b, r.x, acc.x);
+        acc.y = fmaf(b, r.y, acc.y);
+        acc.z = fmaf(b, r.z, acc.z);
+        acc.w = fmaf(b, r.w, acc.w);
+      }
     }
   }
   part[g][c4] = acc;
