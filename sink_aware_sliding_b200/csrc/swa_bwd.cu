@@ -54,11 +54,13 @@ struct BwdCfg {
   static constexpr int QK_STEPS = D / 16;
   static constexpr int PV_STEPS = kBN / 16;
   // shared layout: tiles 0..5 (two fixed, two double-buffered), then D_s, L_s
-  // (128 floats each), then barriers
+  // (128 floats each), the next iterations' D and lse as copied (two buffers of
+  // 128 + 128 floats), then barriers
   static constexpr int OFF_T = 0;
   static constexpr int OFF_DS = 6 * TILE;
   static constexpr int OFF_LS = OFF_DS + 512;
-  static constexpr int OFF_BAR = OFF_LS + 512;
+  static constexpr int OFF_STG = OFF_LS + 512;
+  static constexpr int OFF_BAR = OFF_STG + 2048;
   static constexpr int NBAR = 8;
   static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
   // Each CTA allocates all 512 TMEM columns, so no second CTA may share the SM
@@ -197,6 +199,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     dt = t < a.L ? d_rows[idx] : 0.f;
     l2 = t < a.L ? ba.lse[idx] * 1.4426950408889634f : 0.f;
   };
+  // The same values for a later iteration, copied asynchronously into staging
+  // buffer i & 1 (zero past the sequence's end): a barrier wait that follows loads
+  // into registers would wait for them to land.
+  const uint32_t stg = smem_u32(gbase + C::OFF_STG);
+  auto stage_row = [&](int i) {
+    const int t = it_row0(i) + tid;
+    const bool in = t < a.L;
+    const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + (in ? t : 0);
+    const uint32_t dst = stg + (i & 1) * 1024 + tid * 4;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(d_rows + idx), "r"(in ? 4u : 0u)
+                 : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 512), "l"(ba.lse + idx), "r"(in ? 4u : 0u)
+                 : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
 
   bool ok = true;
   int issued = 0;                                     // iterations whose tiles were requested
@@ -223,7 +240,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       issue(it + 1);
       issued = it + 2;
     }
-    if (it + 1 < n_it) fetch_row(it + 1, next_d, next_l);
+    if (it + 1 < n_it) stage_row(it + 1);
     __syncwarp();
     if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
     if (tid == 0) {
@@ -290,8 +307,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
     // every thread is past this iteration's element-wise step: publish the next row data
     if (it + 1 < n_it) {
-      D_s[tid] = next_d;
-      L_s[tid] = next_l;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      const float* st = reinterpret_cast<const float*>(gbase + C::OFF_STG + ((it + 1) & 1) * 1024);
+      D_s[tid] = st[tid];
+      L_s[tid] = st[128 + tid] * 1.4426950408889634f;
       mbar_arrive(bar(kBarRow));
     }
   }
