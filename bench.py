@@ -489,6 +489,19 @@ def based_linear_flops(w, tokens: int) -> float:
     return 4.0 * w.F * (w.dv + 1) * tokens * w.H
 
 
+def based_linear_bytes(w, tokens: int) -> int:
+    """HBM bytes of a linear-branch prefill: q, k, v read and the bf16 output written
+    (2 (2 dk + dv) + 2 dv bytes per token and head) plus the fp32 final state and
+    normaliser (F (dv + 1) floats per sequence and head)."""
+    return tokens * w.H * (2 * (2 * w.dk + w.dv) + 2 * w.dv) + (tokens // w.L) * w.H * w.F * (w.dv + 1) * 4
+
+
+def based_linear_decode_bytes(w, B: int) -> int:
+    """HBM bytes of one linear-branch decode step: the fp32 state and normaliser read
+    and written, q, k, v read and the bf16 output written."""
+    return B * w.H * (2 * 4 * w.F * (w.dv + 1) + 2 * (2 * w.dk + w.dv) + 2 * w.dv)
+
+
 def bench_based_linear(name, steps, warmup, dev, flush, peaks, sampler):
     """Prefill of the Based linear branch: out [B, L, H, dv] and the final state."""
     import torch
@@ -547,7 +560,7 @@ def bench_based_linear(name, steps, warmup, dev, flush, peaks, sampler):
     # HBM-bound at the roofline: reading q, k, v and writing out and the final state
     # (93.0 MB) takes 14.2 us at the measured copy bandwidth, the FLOPs 11 us at the
     # bf16 tensor peak
-    alg_bytes = w.B * w.L * w.H * (2 * (2 * w.dk + w.dv) + 2 * w.dv) + w.B * w.H * w.F * (w.dv + 1) * 4
+    alg_bytes = based_linear_bytes(w, w.B * w.L)
     gbs = alg_bytes / (ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
@@ -598,7 +611,7 @@ def bench_based_linear_decode(name, steps, warmup, dev, flush, peaks, sampler):
         torch.cuda.synchronize()
     barrier(dev)
     ms = reduce_max(sum(timer.ms()), dev) / steps
-    alg_bytes = B * w.H * (2 * 4 * w.F * (w.dv + 1) + 2 * (2 * w.dk + w.dv) + 2 * w.dv)
+    alg_bytes = based_linear_decode_bytes(w, B)
     gbs = alg_bytes / (ms * 1e-3) / 1e9
 
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))

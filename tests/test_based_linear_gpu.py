@@ -99,6 +99,27 @@ def test_expired_wait_reports_timeout_and_context_survives():
     assert_close(out2, oracle.based_linear_fwd(q, k, v, W.scale), "after timeout")
 
 
+def test_prefill_other_scale():
+    """scale = 0.1 instead of 1/sqrt(dk): sqrt(scale) is no longer a power of two,
+    so the linear features carry their own bf16 rounding."""
+    w = workloads.LinearWorkload("t", B=2, L=300, H=2, dk=W.dk, dv=W.dv)
+    q, k, v = workloads.make_based_linear(w, seed=31)
+    out = torch.empty(2, 300, 2, W.dv, device=DEV)
+    S = torch.full((2, 2, W.F, W.dv), float("nan"), device=DEV)
+    z = torch.full((2, 2, W.F), float("nan"), device=DEV)
+    swa.swa_based_linear_fwd(q.to(DEV), k.to(DEV), v.to(DEV), out, S, z, 0.1)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    assert_close(out, oracle.based_linear_fwd(q, k, v, 0.1), "scale 0.1")
+    wS, wz = oracle.based_linear_state(k, v, 0.1)
+    fk = np.abs(oracle.taylor_features(k, 0.1))
+    c = 2.0 * (300 + 4) * 2.0 ** -24 + 2.0 ** -8
+    bS = c * np.einsum("blhf,blhc->bhfc", fk, np.abs(v.double().numpy())) + 1e-30
+    bz = c * fk.sum(axis=1) + 1e-30
+    assert (np.abs(S.cpu().double().numpy() - wS) <= bS).all()
+    assert (np.abs(z.cpu().double().numpy() - wz) <= bz).all()
+
+
 def test_empty_sequence_writes_a_zero_state():
     q = torch.empty(2, 0, 2, W.dk, dtype=torch.bfloat16)
     v = torch.empty(2, 0, 2, W.dv, dtype=torch.bfloat16)

@@ -33,6 +33,17 @@ def test_workload_flops_match_published_totals():
     assert abs(bench.decode_step_bytes(d, 20000) / 1e9 - 1.0761) < 1e-3
 
 
+def test_linear_branch_counts():
+    w = workloads.LINEAR_WORKLOADS["based_linear"]
+    assert w.F == 273
+    # recurrent form: 4 F (dv + 1) = 70,980 FLOPs per token and head; 8 x 2048 x 16 token-heads
+    assert bench.based_linear_flops(w, w.B * w.L) == 70_980 * 262_144
+    # q, k, v in and out (bf16): 320 bytes per token and head; state and z: 273 x 65 floats per head
+    assert bench.based_linear_bytes(w, w.B * w.L) == 320 * 262_144 + 128 * 273 * 65 * 4 == 92_971_520
+    # decode at B=64: state read and written plus 320 bytes of q, k, v, out per head
+    assert bench.based_linear_decode_bytes(w, 64) == 1024 * (2 * 4 * 273 * 65 + 320) == 145_694_720
+
+
 def _worker(rank, world, port, q):
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
