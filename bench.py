@@ -15,7 +15,8 @@ fused into append and decode, the rotary encoding of the GQA prefill's q and k,
 the Hadamard output projection of the GQA prefill's output (HBM GB/s), and the
 backward pass of the Based-shaped and (at L=8192) the 8B-shaped prefill, and
 the Based hybrid's linear-attention branch (prefill in TFLOP/s of the recurrent
-form's FLOPs, and its recurrent decode step in HBM GB/s).
+form's FLOPs, and its recurrent decode step in HBM GB/s), and the hybrid layer's
+decode (window branch and linear branch side by side, GB/s and tokens/s).
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -654,6 +655,83 @@ def bench_based_linear_decode(name, steps, warmup, dev, flush, peaks, sampler):
     }
 
 
+def bench_hybrid_decode(name, steps, warmup, dev, flush, peaks, sampler):
+    """Decode of a Based-style hybrid layer after a 2048-token prefix: per generated
+    token and sequence, the window branch appends to its 128-slot ring cache and
+    decodes over it (H=16, d=64, no sinks), and the linear branch takes its recurrent
+    step on its fixed-size state (H=16, dk=16, dv=64).  B=64 sequences; the state
+    (72.7 MB) and cache (33.6 MB) fit L2 together, so L2 is flushed before each step."""
+    import torch
+
+    import sink_aware_sliding_b200 as swa
+    import workloads as wl
+    lw = wl.LINEAR_WORKLOADS["based_linear"]
+    B, H, d, W, P = 64, lw.H, 64, 128, 2048
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.SEED)
+    z16 = dict(device=dev, dtype=torch.bfloat16)
+    kc, vc = torch.empty(B, H, W, d, **z16), torch.empty(B, H, W, d, **z16)
+    sk = torch.empty(B, H, 1, d, **z16)                          # unused (no sinks)
+    pk = torch.randn(B, P, H, d, generator=g, device=dev).bfloat16()
+    pv = torch.randn(B, P, H, d, generator=g, device=dev).bfloat16()
+    swa.swa_cache_fill(pk, pv, kc, vc, sk, sk, W, 0)
+    del pk, pv
+    ql, kl, vl = wl.make_based_linear(lw, device=dev, B=B, L=P)
+    S = torch.empty(B, H, lw.F, lw.dv, device=dev)
+    zs = torch.empty(B, H, lw.F, device=dev)
+    swa.swa_based_linear_fwd(ql, kl, vl, torch.empty(B, P, H, lw.dv, **z16), S, zs, lw.scale)
+    del ql, kl, vl
+    n = steps + warmup
+    q = torch.randn(n, B, H, d, generator=g, device=dev).bfloat16()
+    kn = torch.randn(n, B, H, d, generator=g, device=dev).bfloat16()
+    vn = torch.randn(n, B, H, d, generator=g, device=dev).bfloat16()
+    qd = torch.randn(n, B, H, lw.dk, generator=g, device=dev).bfloat16()
+    kd = torch.randn(n, B, H, lw.dk, generator=g, device=dev).bfloat16()
+    vd = torch.randn(n, B, H, lw.dv, generator=g, device=dev).bfloat16()
+    pos = torch.arange(P, P + n, dtype=torch.int32, device=dev).view(-1, 1).expand(-1, B).contiguous()
+    out_w = torch.empty(B, H, d, **z16)
+    out_l = torch.empty(B, H, lw.dv, **z16)
+    lse = torch.empty(B, H, device=dev, dtype=torch.float32)
+    ws = torch.empty(swa.swa_decode_workspace_bytes(B, H, H, d, W, 0), device=dev, dtype=torch.uint8)
+
+    def step(i):
+        swa.swa_cache_append(kn[i], vn[i], pos[i], kc, vc, sk, sk, W, 0)
+        swa.swa_decode(q[i], kc, vc, sk, sk, pos[i], out_w, lse, W, 0, ws)
+        swa.swa_based_linear_decode(qd[i], kd[i], vd[i], S, zs, out_l, lw.scale)
+
+    for i in range(warmup):
+        flush.fill_(1)
+        step(i)
+    torch.cuda.synchronize()
+    timer = Timer(torch)
+    barrier(dev)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(warmup, n):
+            flush.fill_(1)
+            timer(lambda i=i: step(i))
+        torch.cuda.synchronize()
+    barrier(dev)
+    ms = reduce_max(sum(timer.ms()), dev) / steps
+    if swa.swa_device_error() != 0:
+        raise RuntimeError("hybrid decode reported a device wait timeout")
+    # HBM bytes per step: the window cache read (k and v), the appended rows, q and out
+    # of the window branch, and the linear step's state and vectors
+    alg_bytes = (2 * B * H * W * d * 2 + 2 * B * H * d * 2 + 2 * B * H * d * 2 + 8 * B * H
+                 + based_linear_decode_bytes(lw, B))
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"], "traffic": None,
+            "algorithmic_bytes_per_launch": alg_bytes}
+    return {
+        "config": {"workload": name, "kind": "hybrid_decode", "B": B, "H": H, "window": W, "d": d,
+                   "linear_dk": lw.dk, "linear_dv": lw.dv, "prefix": P},
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
+        "tokens_per_s": round(B / (ms * 1e-3), 1), "roofline": roof,
+        "e2e": None, "gpu_launches": 4 * steps, "l2": "flushed between steps (512 MiB write)",
+    }
+
+
 def bench_bwd(name, steps, warmup, dev, flush, peaks, sampler):
     """Backward pass (dq, dk, dv) of a prefill workload; FLOPs: five products of 2*d per
     visible pair and query head (S, dP, dV, dK, dQ), i.e. 2.5x the forward's."""
@@ -978,7 +1056,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
     ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj,"
-                    "bwd_based_local,bwd_gqa8b_L8192,based_linear,based_linear_decode")
+                    "bwd_based_local,bwd_gqa8b_L8192,based_linear,based_linear_decode,hybrid_decode")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -1036,6 +1114,8 @@ def main():
             results[n] = bench_based_linear(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         elif n == "based_linear_decode":
             results[n] = bench_based_linear_decode(n, args.steps, args.warmup, dev, flush, peaks, sampler)
+        elif n == "hybrid_decode":
+            results[n] = bench_hybrid_decode(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         else:
             results[n] = bench_prefill(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         torch.cuda.empty_cache()
