@@ -281,11 +281,22 @@ def swa_based_linear_fwd(q, k, v, out, state=None, zsum=None, scale=None, stream
     """Causal Taylor linear attention: q, k [B, L, H, dk], v [B, L, H, dv] bf16 -> out (bf16 or
     float32); state [B, H, F, dv] / zsum [B, H, F] float32, if given, receive the final state."""
     import torch
+    _need(q.dim() == 4, "q [B, L, H, dk]")
     B, L, H, dk = q.shape
     dv = v.shape[-1]
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t.dtype == torch.bfloat16 and t.is_contiguous(), f"{n} bf16 contiguous")
+    _need(k.shape == q.shape, "k shape == q shape")
+    _need(v.dim() == 4 and v.shape[:3] == q.shape[:3], "v [B, L, H, dv]")
+    _need(out.shape == v.shape and out.is_contiguous() and out.dtype in (torch.bfloat16, torch.float32),
+          "out [B, L, H, dv] bf16 or float32, contiguous")
     _need((state is None) == (zsum is None), "state and zsum together")
+    if state is not None:
+        F = 1 + dk + dk * dk
+        _need(state.shape == (B, H, F, dv) and state.dtype == torch.float32 and state.is_contiguous(),
+              "state [B, H, F, dv] float32 contiguous")
+        _need(zsum.shape == (B, H, F) and zsum.dtype == torch.float32 and zsum.is_contiguous(),
+              "zsum [B, H, F] float32 contiguous")
     code = SWA_DTYPE_F32 if out.dtype == torch.float32 else SWA_DTYPE_BF16
     st = _load().swa_based_linear_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(zsum), B, L, H, dk, dv,
                                       ctypes.c_float(scale if scale is not None else 1.0 / math.sqrt(dk)), code,
@@ -297,8 +308,19 @@ def swa_based_linear_decode(q, k, v, state, zsum, out, scale=None, stream=None) 
     """One token per sequence: q, k [B, H, dk], v [B, H, dv] bf16; state/zsum float32 updated
     in place; out [B, H, dv]."""
     import torch
+    _need(q.dim() == 3, "q [B, H, dk]")
     B, H, dk = q.shape
     dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t.dtype == torch.bfloat16 and t.is_contiguous(), f"{n} bf16 contiguous")
+    _need(k.shape == q.shape and v.dim() == 3 and v.shape[:2] == q.shape[:2], "k [B, H, dk], v [B, H, dv]")
+    F = 1 + dk + dk * dk
+    _need(state.shape == (B, H, F, dv) and state.dtype == torch.float32 and state.is_contiguous(),
+          "state [B, H, F, dv] float32 contiguous")
+    _need(zsum.shape == (B, H, F) and zsum.dtype == torch.float32 and zsum.is_contiguous(),
+          "zsum [B, H, F] float32 contiguous")
+    _need(out.shape == v.shape and out.is_contiguous() and out.dtype in (torch.bfloat16, torch.float32),
+          "out [B, H, dv] bf16 or float32, contiguous")
     code = SWA_DTYPE_F32 if out.dtype == torch.float32 else SWA_DTYPE_BF16
     st = _load().swa_based_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(zsum), _ptr(out), B, H, dk, dv,
                                          ctypes.c_float(scale if scale is not None else 1.0 / math.sqrt(dk)), code,

@@ -112,3 +112,28 @@ def test_based_linear_argument_checks(lib):
     assert dec(dk=8) == swa.SWA_ERR_UNSUPPORTED
     assert dec() == swa.SWA_ERR_INVALID_ARG
     assert dec(B=0) == swa.SWA_OK
+
+
+def test_based_linear_binding_checks_shapes(lib):
+    # shape and dtype checks happen in the binding before any device work (CPU tensors)
+    import torch
+    bf = dict(dtype=torch.bfloat16)
+    q = torch.zeros(1, 8, 2, 16, **bf)
+    v = torch.zeros(1, 8, 2, 64, **bf)
+    out = torch.zeros(1, 8, 2, 64, **bf)
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_fwd(q, torch.zeros(1, 8, 2, 8, **bf), v, out)          # k shape
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_fwd(q, q, v, torch.zeros(1, 8, 2, 32, **bf))          # out shape
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_fwd(q, q, v, out, torch.zeros(1, 2, 100, 64), torch.zeros(1, 2, 100))
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_fwd(q, q, v, out, torch.zeros(1, 2, 273, 64), None)
+    qd = torch.zeros(1, 2, 16, **bf)
+    vd = torch.zeros(1, 2, 64, **bf)
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_decode(qd, qd, vd, torch.zeros(1, 2, 273, 64, dtype=torch.float64),
+                                    torch.zeros(1, 2, 273), torch.zeros(1, 2, 64))
+    with pytest.raises(ValueError):
+        swa.swa_based_linear_decode(qd, qd, vd, torch.zeros(1, 2, 273, 64), torch.zeros(1, 2, 272),
+                                    torch.zeros(1, 2, 64))
