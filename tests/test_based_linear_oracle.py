@@ -106,3 +106,24 @@ def test_planted_mistake_fails_a_pin(mistake):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, mistake
+
+
+def test_hand_worked_example():
+    """tests/golden/hand_based_linear_d2.json: a two-token prefill and one decode step
+    with dk = 2, dv = 1, worked by hand (the derivation is in the file)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_based_linear_d2.json")))
+    s = g["scale"]
+    q = np.array(g["q"])[None, :, None, :]
+    k = np.array(g["k"])[None, :, None, :]
+    v = np.array(g["v"])[None, :, None, :]
+    np.testing.assert_allclose(oracle.based_linear_fwd(q, k, v, s)[0, :, 0], g["out"], rtol=1e-14)
+    S, z = oracle.based_linear_state(k, v, s)
+    np.testing.assert_allclose(S[0, 0], g["S"], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(z[0, 0], g["z"], rtol=1e-14, atol=1e-14)
+    out, S2, z2 = oracle.based_linear_decode(np.array(g["q_next"])[None, None], np.array(g["k_next"])[None, None],
+                                             np.array(g["v_next"])[None, None], S, z, s)
+    np.testing.assert_allclose(out[0, 0], g["out_next"], rtol=1e-14)
+    np.testing.assert_allclose(S2[0, 0], g["S_next"], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(z2[0, 0], g["z_next"], rtol=1e-14, atol=1e-14)
