@@ -2,21 +2,23 @@
 """Benchmark of sink-aware sliding-window attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl swa|reference]
-                    [--workloads based_local,gqa8b_prefill,packed_long,decode]
+                    [--workloads packed_long,gqa8b_prefill,based_local,decode,...]
 
 Prints ONE JSON line on rank 0.  The headline (`value`) is the prefill
-throughput in TFLOP/s of the Based-style local-window workload (B=8, H=16,
-L=2048, d=64, window 128), counting 4*d FLOPs per visible (query, key) pair.
-The same line carries, under "workloads", the other workloads measured the
-same way: the 8B-shaped GQA prefill and the packed long-context prefill
-(TFLOP/s against the tensor roofline) and the ring-buffer decode (HBM GB/s and
-tokens/s against the HBM roofline), the same decode with the rotary encoding
-fused into append and decode, the rotary encoding of the GQA prefill's q and k,
-the Hadamard output projection of the GQA prefill's output (HBM GB/s), and the
-backward pass of the Based-shaped and (at L=8192) the 8B-shaped prefill, and
-the Based hybrid's linear-attention branch (prefill in TFLOP/s of the recurrent
-form's FLOPs, and its recurrent decode step in HBM GB/s), and the hybrid layer's
-decode (window branch and linear branch side by side, GB/s and tokens/s).
+throughput in TFLOP/s of the long-context packed prefill (sequences of 131072,
+65536, 16384 and 1000 tokens, Hq=32, Hkv=8, d=128, window 2048, 4 sinks), the
+largest workload that fits one GPU, counting 4*d FLOPs per visible (query, key)
+pair, against the bf16 tensor roofline.  The same line carries, under
+"workloads", the other workloads measured the same way: the 8B-shaped GQA
+prefill and the Based-style local-window prefill (TFLOP/s against the tensor or
+the HBM roofline), the ring-buffer decode at B=64 and B=1 (HBM GB/s and
+tokens/s), the same decode with the rotary encoding fused into append and
+decode, the rotary encoding of the GQA prefill's q and k, the Hadamard output
+projection of the GQA prefill's output (HBM GB/s), the backward pass of the
+Based-shaped and (at L=8192) the 8B-shaped prefill, the Based hybrid's
+linear-attention branch (prefill in TFLOP/s of the recurrent form's FLOPs, and
+its recurrent decode step in HBM GB/s), and the hybrid layer's decode (window
+branch and linear branch side by side, GB/s and tokens/s).
 
 Timing: inputs are generated on the device and stay resident; W untimed
 warm-up steps; K timed steps between a barrier plus device synchronisation on
@@ -30,8 +32,13 @@ same workload on its own GPU, times are reduced with a max over ranks.
 memory: each step copies its inputs host->device, runs the kernel(s) and
 copies the outputs back, all inside the timed region.
 
-`--impl reference` times the fp64 CPU oracle on the host cores instead (the
-reference arm); it runs on rank 0 only.
+`cpu_baseline` is the fp64 oracle on the host cores: over the headline's
+sampled query rows (the sink and window edges, query-block edges, the last 64
+rows and 256 seeded random rows of every sequence, all heads), as a rate on
+the sample's visible pairs with the whole workload's time extrapolated from it;
+the Based-style prefill in full; the GQA prefill on sampled rows; the decode on
+four full steps.  `--impl reference` times the same oracle on the headline's
+sample (the reference arm); it runs on rank 0 only.
 """
 from __future__ import annotations
 
@@ -50,7 +57,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "sink-SWA prefill TFLOP/s (visible pairs) & decode HBM GB/s, % of B200 roofline"
-HEADLINE = "based_local"
+HEADLINE = "packed_long"
 L2_FLUSH_BYTES = 512 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -896,47 +903,157 @@ def bench_decode(name, steps, warmup, dev, peaks, sampler):
 
 
 # --------------------------------------------------------------------------- oracle (CPU)
-def oracle_rate(name: str, min_seconds: float = 10.0, max_seconds: float = 30.0):
-    """The fp64 oracle on the host cores over a bounded sample of the workload.
-    Returns (TFLOP/s, cores, sample description)."""
+def _gen_device():
+    """Where the seeded inputs are drawn: on the GPU when there is one (the same values the
+    GPU arm measures), else on the host (same recipe, different generator stream)."""
+    import torch
+    return torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+
+
+def _f64_host(x):
+    import torch
+    return x.detach().to("cpu").to(torch.float64).numpy()
+
+
+def oracle_prefill_sample(name: str):
+    """Host copies (float64) of a prefill workload's sampled query rows and of the keys and
+    values they read: per sequence, all heads of the rows {0 .. s+1, w-2 .. w+s+1, the
+    edges of four 128-row query blocks, the last 64 rows, 256 random rows (seed 1)}, which
+    include each sequence's first row.  Returns (parts, pairs, total_pairs) with parts a
+    list of (q_rows, rows, k, v) per sequence, pairs the visible (row, head) pairs the
+    sample holds and total_pairs those of the whole workload."""
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    dev = _gen_device()
+    if w.kind == "varlen":
+        q, k, v, cu = wl.make_varlen(w, device=dev)
+        seqs = [(q[cu[i]:cu[i] + n], k[cu[i]:cu[i] + n], v[cu[i]:cu[i] + n]) for i, n in enumerate(w.seqlens)]
+    else:
+        q, k, v = wl.make_prefill(w, device=dev)
+        seqs = [(q[b], k[b], v[b]) for b in range(w.B)]
+    parts, pairs, total = [], 0, 0
+    for qs, ks, vs in seqs:
+        n = qs.shape[0]
+        rows = wl.sample_rows(n, w.window, w.n_sink, n_random=256, seed=1)
+        parts.append((_f64_host(qs[rows]), rows, _f64_host(ks), _f64_host(vs)))
+        pairs += w.Hq * sum(min(t + 1, w.window) + min(max(t - w.window + 1, 0), w.n_sink) for t in rows)
+        total += w.Hq * visible_pairs(n, w.window, w.n_sink)
+    del q, k, v, seqs
+    return parts, pairs, total
+
+
+def oracle_prefill_pass(name: str, parts) -> float:
+    """One pass of the oracle over a sample; returns the seconds it took."""
     import oracle
     import workloads as wl
     w = wl.WORKLOADS[name]
-    cores = oracle.num_threads()
-    if w.kind == "prefill" and w.B * w.L * w.Hq <= 8 * 2048 * 16:
-        q, k, v = wl.make_prefill(w)
-        flops = prefill_flops(w, [w.L] * w.B)
-        sample = f"whole workload ({w.B} sequences x {w.L} rows x {w.Hq} heads), repeated"
-        passes, t0 = 0, time.perf_counter()
-        while True:
-            oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
-            passes += 1
-            dt = time.perf_counter() - t0
-            if dt >= min_seconds or dt * (passes + 1) / passes > max_seconds:
-                break
-        return flops * passes / dt / 1e12, cores, f"{sample} {passes} times in {dt:.1f} s"
-    raise ValueError(f"no CPU sample defined for {name}")
+    t0 = time.perf_counter()
+    for q_rows, rows, k, v in parts:
+        oracle.swa_rows(q_rows, rows, k, v, w.window, w.n_sink, w.scale)
+    return time.perf_counter() - t0
+
+
+def oracle_prefill_rate(name: str, min_seconds: float = 10.0, max_seconds: float = 30.0) -> dict:
+    """The fp64 oracle on the host cores over the sampled rows of a prefill workload:
+    TFLOP/s on the sample's visible pairs (4 d FLOPs per pair and head), and the time
+    the whole workload would take at that rate (extrapolated, not measured)."""
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    parts, pairs, total = oracle_prefill_sample(name)
+    secs, passes = 0.0, 0
+    while True:
+        secs += oracle_prefill_pass(name, parts)
+        passes += 1
+        if secs >= min_seconds or secs * (passes + 1) / passes > max_seconds:
+            break
+    flops = 4 * w.d * pairs * passes
+    rate = flops / secs
+    n_rows = sum(len(p[1]) for p in parts)
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{n_rows} sampled query rows x {w.Hq} heads over {len(parts)} sequence(s) "
+                       f"({pairs} visible pairs), {passes} passes in {secs:.1f} s; full workload "
+                       f"extrapolated at the sample's per-pair rate"),
+            "pairs_per_s": round(pairs * passes / secs, 1),
+            "extrapolated_full_s": round(4 * w.d * total / rate, 2)}
+
+
+def oracle_decode_rate(name: str, steps: int = 4) -> dict:
+    """The fp64 oracle on the host cores for ``steps`` consecutive decode steps of the
+    decode workload (every sequence and head), reported per step.  For each sequence the
+    keys and values the steps can see (the sinks and positions prefix-w+1 .. prefix+steps-1)
+    are handed to the oracle as one short sequence in which step i is row s + w - 1 + i;
+    without positional terms in the scores this is the same visible set, the same
+    arithmetic and the same result."""
+    import torch
+
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    if w.rope_base > 0:
+        raise ValueError("the per-step oracle timing covers the decode without rotary encoding")
+    dev = _gen_device()
+    di = wl.make_decode(w, device=dev, steps=steps)
+    P, W, S = w.prefix, w.window, w.n_sink
+    secs = 0.0
+    for b in range(w.B):
+        k = torch.cat([di.prefix_k[b, :S], di.prefix_k[b, P - W + 1:], di.k_new[:, b]], dim=0)
+        v = torch.cat([di.prefix_v[b, :S], di.prefix_v[b, P - W + 1:], di.v_new[:, b]], dim=0)
+        kh, vh, qh = _f64_host(k), _f64_host(v), _f64_host(di.q[:, b])
+        rows = [S + W - 1 + i for i in range(steps)]
+        t0 = time.perf_counter()
+        oracle.swa_rows(qh, rows, kh, vh, W, S, w.scale)
+        secs += time.perf_counter() - t0
+    del di
+    per_step = secs / steps
+    keys = min(P + 1, W) + min(max(P - W + 1, 0), S)
+    return {"value": round(decode_step_bytes(w, P) / per_step / 1e9, 4), "unit": "GB/s",
+            "ms_per_step": round(per_step * 1e3, 2), "tokens_per_s": round(w.B / per_step, 2),
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{steps} full decode steps (B={w.B} x {w.Hq} heads, {keys} visible keys each) "
+                       f"after the {P}-token prefix, {secs:.3f} s")}
+
+
+def oracle_full_rate(name: str, min_seconds: float = 5.0, max_seconds: float = 30.0) -> dict:
+    """The fp64 oracle on the host cores over a whole (small) prefill workload, repeated."""
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    dev = _gen_device()
+    q, k, v = (_f64_host(x) for x in wl.make_prefill(w, device=dev))
+    flops = prefill_flops(w, [w.L] * w.B)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or dt * (passes + 1) / passes > max_seconds:
+            break
+    return {"value": round(flops * passes / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"whole workload ({w.B} sequences x {w.L} rows x {w.Hq} heads), {passes} passes in {dt:.1f} s"}
 
 
 def reference_arm(args):
-    """The fp64 oracle as the reference arm: each step is one pass over a bounded sample."""
+    """The fp64 oracle as the reference arm: each step is one pass over the headline
+    workload's sampled rows (the same sample as the GPU arm's cpu_baseline)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import oracle
     import workloads as wl
     w = wl.WORKLOADS[HEADLINE]
-    q, k, v = wl.make_prefill(w, B=1)
-    flops = prefill_flops(w, [w.L])
+    parts, pairs, total = oracle_prefill_sample(HEADLINE)
     cores = oracle.num_threads()
     for _ in range(args.warmup):
-        oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.swa_fwd(q, k, v, w.window, w.n_sink, w.scale)
-    dt = time.perf_counter() - t0
+        oracle_prefill_pass(HEADLINE, parts)
+    dt = sum(oracle_prefill_pass(HEADLINE, parts) for _ in range(args.steps))
+    flops = 4 * w.d * pairs
     val = flops * args.steps / dt / 1e12
-    sample = f"1 of {w.B} sequences ({w.L} rows x {w.Hq} heads) per step"
+    n_rows = sum(len(p[1]) for p in parts)
+    sample = (f"{n_rows} sampled query rows x {w.Hq} heads over {len(parts)} sequences ({pairs} visible "
+              f"pairs) per step; full workload extrapolated at this rate: "
+              f"{4 * w.d * total / (flops * args.steps / dt):.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -1055,8 +1172,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["swa", "reference"], default="swa")
-    ap.add_argument("--workloads", default="based_local,gqa8b_prefill,packed_long,decode,decode_rope,rope_qk_gqa8b,hadamard_proj,"
-                    "bwd_based_local,bwd_gqa8b_L8192,based_linear,based_linear_decode,hybrid_decode")
+    ap.add_argument("--workloads", default="packed_long,gqa8b_prefill,based_local,decode,decode_b1,decode_rope,"
+                    "rope_qk_gqa8b,hadamard_proj,bwd_based_local,bwd_gqa8b_L8192,based_linear,based_linear_decode,"
+                    "hybrid_decode")
     ap.add_argument("--decode-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -1088,21 +1206,30 @@ def main():
     import sink_aware_sliding_b200 as swa
     swa.library()
 
-    # CPU baseline first, before any large device allocation (rank 0, one GPU only).
-    cpu = None
+    # CPU baselines first, while the GPU is idle (rank 0, one GPU only): the oracle over the
+    # headline's sampled rows, and for the other prefill and decode workloads likewise.
+    cpu, cpu_other = None, {}
+    names = [n for n in args.workloads.split(",") if n]
+    if HEADLINE not in names:
+        names.insert(0, HEADLINE)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, cores, sample = oracle_rate(HEADLINE)
-        cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = oracle_prefill_rate(HEADLINE)
+        for n in names:
+            if n == "based_local":
+                cpu_other[n] = oracle_full_rate(n)
+            elif n == "gqa8b_prefill":
+                cpu_other[n] = oracle_prefill_rate(n, min_seconds=5.0)
+            elif n in ("decode", "decode_b1"):
+                cpu_other[n] = oracle_decode_rate(n)
+        import torch as _t
+        _t.cuda.empty_cache()
 
     peaks = load_peaks()
     sampler = ClockSampler(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    names = [n for n in args.workloads.split(",") if n]
-    if HEADLINE not in names:
-        names.insert(0, HEADLINE)
     results = {}
     for n in names:
-        if n in ("decode", "decode_rope"):
+        if n in ("decode", "decode_rope", "decode_b1"):
             results[n] = bench_decode(n, args.decode_tokens, args.warmup, dev, peaks, sampler)
         elif n.startswith("bwd_"):
             results[n] = bench_bwd(n, max(3, args.steps // 4), args.warmup, dev, flush, peaks, sampler)
@@ -1118,6 +1245,8 @@ def main():
             results[n] = bench_hybrid_decode(n, args.steps, args.warmup, dev, flush, peaks, sampler)
         else:
             results[n] = bench_prefill(n, args.steps, args.warmup, dev, flush, peaks, sampler)
+        if n in cpu_other:
+            results[n]["cpu_baseline"] = cpu_other[n]
         torch.cuda.empty_cache()
 
     head = results[HEADLINE]

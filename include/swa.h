@@ -21,6 +21,10 @@
  *     legacy default stream).  The return value reports argument errors
  *     (nothing launched) and launch errors only; a device-side wait that ran
  *     past its time limit is reported through swa_device_error.
+ *   - The library keeps, per device, addresses it looked up once (its error
+ *     word, and swa_decode_noalloc's scratch array).  It must not be used on a
+ *     device after cudaDeviceReset, or after its primary context was destroyed
+ *     and created again, within the same process.
  *   - bf16 is IEEE bfloat16 stored as uint16; f32 is IEEE binary32.
  *   - Accumulation is fp32.  In the bf16 path the softmax numerators P are
  *     rounded to bf16 (round-to-nearest-even) before the P.V product and the
@@ -137,6 +141,18 @@ int swa_decode(const void* q, const void* kcache, const void* vcache,
                void* workspace, size_t workspace_bytes, swa_stream_t stream);
 
 /*
+ * swa_decode with a choice of output type: out_dtype SWA_DTYPE_BF16 writes out
+ * as bf16 (exactly swa_decode), SWA_DTYPE_BF16_F32OUT writes it as float32 (the
+ * same arithmetic without the final rounding, for checking the kernels'
+ * arithmetic on its own).  Anything else is SWA_ERR_INVALID_ARG.
+ */
+int swa_decode_ex(const void* q, const void* kcache, const void* vcache,
+                  const void* sink_k, const void* sink_v, const int32_t* pos,
+                  void* out, float* lse,
+                  int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
+                  int out_dtype, void* workspace, size_t workspace_bytes, swa_stream_t stream);
+
+/*
  * swa_decode without a workspace argument, for callers that cannot allocate
  * device memory: code that runs inside a host framework which owns every
  * device allocation (a serving engine with a preallocated arena, a plugin in
@@ -153,7 +169,13 @@ int swa_decode(const void* q, const void* kcache, const void* vcache,
  * for the 64 x 32 x 8 x 128 decode workload the need is about 3.5 MiB.
  * The first call on each device looks up that device's address of the array
  * (cudaGetSymbolAddress, with the device current); make that first call
- * before any stream capture.  All calls on a device share the one array and
+ * before any stream capture.  With CUDA's lazy module loading (the default
+ * since CUDA 12.2) the library's device code, this array included, is loaded
+ * onto a device when the library is first used there, which can be that first
+ * call: a caller that may not allocate after start-up makes one call (any
+ * valid decode) at start-up, or sets CUDA_MODULE_LOADING=EAGER.  The argument
+ * checks of swa_decode come first (SWA_ERR_INVALID_ARG / SWA_ERR_UNSUPPORTED as
+ * there), then the size check against the array.  All calls on a device share the one array and
  * it keeps whatever the last call left there; every value a call reads was
  * written earlier in the same call, so nothing needs clearing, but calls
  * whose work overlaps on the GPU (different streams, or different host
@@ -283,6 +305,9 @@ const char* swa_status_string(int status);
  * memory).  Returns SWA_ERR_CUDA if the synchronisation itself failed.
  */
 int swa_device_error(swa_stream_t stream);
+
+/* The same call under a second name: reads and clears the device error word. */
+int swa_debug_error_word(swa_stream_t stream);
 
 /*
  * Time limit, in nanoseconds, of every device-side barrier wait launched after

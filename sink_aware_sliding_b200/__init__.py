@@ -38,6 +38,7 @@ EXPORTS = (
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
     "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope", "swa_bwd",
     "swa_based_linear_state_features", "swa_based_linear_fwd", "swa_based_linear_decode",
+    "swa_decode_ex", "swa_debug_error_word",
 )
 
 _lib = None
@@ -64,6 +65,7 @@ def _load():
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = SZ
     lib.swa_decode.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_decode_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, SZ, P]
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.swa_hadamard_proj.argtypes = [P, P, P, P, LL, I, I, P]
     D = ctypes.c_double
@@ -77,11 +79,12 @@ def _load():
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     lib.swa_device_error.argtypes = [P]
+    lib.swa_debug_error_word.argtypes = [P]
     lib.swa_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
     lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
-                 "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
+                 "swa_decode_ex", "swa_debug_error_word", "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
                  "swa_decode_rope", "swa_bwd", "swa_based_linear_state_features", "swa_based_linear_fwd",
                  "swa_based_linear_decode",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
@@ -222,14 +225,19 @@ def swa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, window: int, n
 
 def swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,
                workspace, scale=None, stream=None) -> None:
-    """One decode step; q [B, Hq, d] bf16 at positions pos; writes out [B, Hq, d] and lse [B, Hq]."""
+    """One decode step; q [B, Hq, d] bf16 at positions pos; writes out [B, Hq, d] and lse [B, Hq].
+    out is bf16 (swa_decode) or float32 (swa_decode_ex with a float32 output)."""
+    import torch
     B, Hq, d = q.shape
     Hkv = kcache.shape[1]
-    st = _load().swa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(sink_k), _ptr(sink_v),
-                            _ptr(pos), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window), int(n_sink),
-                            _scale(scale, d), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                            _stream(stream))
-    _check(st, "swa_decode")
+    _need(out.dtype in (torch.bfloat16, torch.float32), "out bf16 or float32")
+    args = (_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(sink_k), _ptr(sink_v), _ptr(pos), _ptr(out), _ptr(lse),
+            B, Hq, Hkv, d, int(window), int(n_sink), _scale(scale, d))
+    ws = (_ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if out.dtype == torch.float32:
+        _check(_load().swa_decode_ex(*args, SWA_DTYPE_BF16_F32OUT, *ws), "swa_decode_ex")
+    else:
+        _check(_load().swa_decode(*args, *ws), "swa_decode")
 
 
 def swa_decode_rope(q, kcache, vcache, sink_k, sink_v, pos, out, lse, window: int, n_sink: int,
@@ -347,6 +355,10 @@ def swa_hadamard_proj(y, alpha, beta, z, stream=None) -> None:
 
 def swa_device_error(stream=None) -> int:
     return _load().swa_device_error(_stream(stream))
+
+
+def swa_debug_error_word(stream=None) -> int:
+    return _load().swa_debug_error_word(_stream(stream))
 
 
 def swa_set_wait_timeout_ns(ns: int) -> int:

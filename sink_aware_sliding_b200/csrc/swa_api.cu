@@ -159,15 +159,22 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-int decode_grid(DeviceInfo* dev, int d, int B, int* grid) {
+// Split-K decode grid: one warp per kDecodeKeysPerWarp keys of the largest
+// possible visible set (every segment holds at most window + n_sink keys; the
+// positions themselves are on the device), and never more CTAs than fill the GPU.
+constexpr long long kDecodeKeysPerWarp = 32;
+int decode_grid(DeviceInfo* dev, int d, int B, int Hkv, int window, int n_sink, int* grid) {
   const int idx = d == 128 ? 1 : 0;
   if (dev->decode_ctas_per_sm[idx] == 0) {
     int c = 0;
     if (swa::decode_occupancy(d, 4096, &c) != cudaSuccess || c <= 0) return SWA_ERR_CUDA;
     dev->decode_ctas_per_sm[idx] = c;
   }
-  (void)B;
-  *grid = dev->sms * dev->decode_ctas_per_sm[idx];
+  const long long full = static_cast<long long>(dev->sms) * dev->decode_ctas_per_sm[idx];
+  const long long max_keys = static_cast<long long>(B) * Hkv * (static_cast<long long>(window) + n_sink);
+  const long long warps = (max_keys + kDecodeKeysPerWarp - 1) / kDecodeKeysPerWarp;
+  const long long wpc = swa::decode_threads() / 32;
+  *grid = static_cast<int>(std::max(1LL, std::min(full, (warps + wpc - 1) / wpc)));
   return SWA_OK;
 }
 
@@ -260,25 +267,42 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int window, int
   DeviceInfo* dev = nullptr;
   if (device_info(&dev) != SWA_OK) return 0;
   int grid = 0;
-  if (decode_grid(dev, d, B, &grid) != SWA_OK) return 0;
+  if (decode_grid(dev, d, B, Hkv, window, n_sink, &grid) != SWA_OK) return 0;
   const size_t n_warps = static_cast<size_t>(grid) * (swa::decode_threads() / 32);
   const size_t slots = n_warps + static_cast<size_t>(B) * Hkv;
   return slots * swa::decode_partial_floats(Hq / Hkv, d) * sizeof(float);
 }
 
-static int run_decode(const void* q, const void* kcache, const void* vcache, const void* sink_k,
-                      const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
-                      int Hkv, int d, int window, int n_sink, float scale, void* workspace,
-                      size_t workspace_bytes, const swa::RopeTable* rope, swa_stream_t stream) {
+}  // extern "C"
+
+namespace swa {
+
+int decode_args_status(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                       const void* sink_v, const int32_t* pos, const void* out, const float* lse, int B,
+                       int Hq, int Hkv, int d, int window, int n_sink, float scale, int out_dtype) {
   int st = decode_shape_ok(B, Hq, Hkv, d, window, n_sink);
   if (st != SWA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (out_dtype != SWA_DTYPE_BF16 && out_dtype != SWA_DTYPE_BF16_F32OUT) return SWA_ERR_INVALID_ARG;
   if (B == 0) return SWA_OK;
   if (!q || !pos || !out || !aligned16(q) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(pos) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return SWA_ERR_INVALID_ARG;
-  st = check_cache(B, Hkv, d, window, n_sink, kcache, vcache, sink_k, sink_v);
+  return check_cache(B, Hkv, d, window, n_sink, kcache, vcache, sink_k, sink_v);
+}
+
+}  // namespace swa
+
+extern "C" {
+
+static int run_decode(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                      const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
+                      int Hkv, int d, int window, int n_sink, float scale, int out_dtype, void* workspace,
+                      size_t workspace_bytes, const swa::RopeTable* rope, swa_stream_t stream) {
+  int st = swa::decode_args_status(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window,
+                                   n_sink, scale, out_dtype);
   if (st != SWA_OK) return st;
+  if (B == 0) return SWA_OK;
   const size_t need = swa_decode_workspace_bytes(B, Hq, Hkv, d, window, n_sink);
   if (need == 0) return SWA_ERR_CUDA;
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -286,7 +310,7 @@ static int run_decode(const void* q, const void* kcache, const void* vcache, con
   DeviceInfo* dev = nullptr;
   if ((st = device_info(&dev)) != SWA_OK) return st;
   int grid = 0;
-  if ((st = decode_grid(dev, d, B, &grid)) != SWA_OK) return st;
+  if ((st = decode_grid(dev, d, B, Hkv, window, n_sink, &grid)) != SWA_OK) return st;
   swa::DecodeArgs a{};
   a.q = q;
   a.kcache = kcache;
@@ -305,6 +329,7 @@ static int run_decode(const void* q, const void* kcache, const void* vcache, con
   a.S = n_sink;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.n_warps = grid * (swa::decode_threads() / 32);
+  a.out_f32 = out_dtype == SWA_DTYPE_BF16_F32OUT ? 1 : 0;
   cudaError_t e = swa::launch_decode(a, d, grid, swa::decode_threads(),
                                      reinterpret_cast<cudaStream_t>(stream), rope);
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
@@ -315,7 +340,15 @@ int swa_decode(const void* q, const void* kcache, const void* vcache, const void
                int Hkv, int d, int window, int n_sink, float scale, void* workspace,
                size_t workspace_bytes, swa_stream_t stream) {
   return run_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
-                    scale, workspace, workspace_bytes, nullptr, stream);
+                    scale, SWA_DTYPE_BF16, workspace, workspace_bytes, nullptr, stream);
+}
+
+int swa_decode_ex(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                  const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq, int Hkv,
+                  int d, int window, int n_sink, float scale, int out_dtype, void* workspace,
+                  size_t workspace_bytes, swa_stream_t stream) {
+  return run_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
+                    scale, out_dtype, workspace, workspace_bytes, nullptr, stream);
 }
 
 static bool rope_base_ok(double base) { return base > 0.0 && std::isfinite(base); }
@@ -328,7 +361,7 @@ int swa_decode_rope(const void* q, const void* kcache, const void* vcache, const
   swa::RopeTable rt;
   swa::make_rope_table(rope_base, d, &rt);
   return run_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
-                    scale, workspace, workspace_bytes, &rt, stream);
+                    scale, SWA_DTYPE_BF16, workspace, workspace_bytes, &rt, stream);
 }
 
 int swa_rope_qk(void* q, void* k, const int32_t* positions, long long n_tokens, int Hq, int Hkv, int d,
@@ -510,6 +543,8 @@ int swa_device_error(swa_stream_t stream) {
     return SWA_ERR_CUDA;
   return v;
 }
+
+int swa_debug_error_word(swa_stream_t stream) { return swa_device_error(stream); }
 
 unsigned long long swa_set_wait_timeout_ns(unsigned long long ns) { return g_timeout_ns.exchange(ns); }
 

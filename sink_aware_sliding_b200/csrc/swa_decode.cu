@@ -71,6 +71,14 @@ __device__ __forceinline__ uint32_t pair(const uint4& a, const uint4& b, int e) 
   return __byte_perm(word(a, e >> 1), word(b, e >> 1), (e & 1) ? 0x7632 : 0x5410);
 }
 
+// Number of pieces the K concatenated keys are cut into: one per warp of the grid,
+// but no more than one per kMinPieceKeys keys, so that no piece is empty (each piece
+// has at least one key whenever pieces <= K) and short contexts are not spread thin.
+constexpr long long kMinPieceKeys = 16;
+__device__ __forceinline__ long long effective_pieces(long long K, long long n_warps) {
+  return max(1LL, min(n_warps, (K + kMinPieceKeys - 1) / kMinPieceKeys));
+}
+
 // Binary search: the batch b whose segments [pre[b]*Hkv, pre[b+1]*Hkv) hold key x.
 __device__ __forceinline__ int find_batch(const long long* pre, int B, long long x, int Hkv) {
   int lo = 0, hi = B - 1;
@@ -124,8 +132,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
   __syncthreads();
 
   const long long K = s_pre[B] * Hkv;
-  const long long Wn = a.n_warps;
+  const long long Wn = effective_pieces(K, a.n_warps);
   const long long wid = static_cast<long long>(blockIdx.x) * (kDecodeThreads / 32) + (threadIdx.x >> 5);
+  if (wid >= Wn) return;                 // fewer keys than the grid was sized for: idle warp
   long long x = wid * K / Wn;
   const long long x_end = (wid + 1) * K / Wn;
   const size_t part_floats = static_cast<size_t>(G) * (D + 2);
@@ -288,58 +297,117 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 }
 
-// One CTA per (b, kvh) segment: combine the partials of the warps that covered it.
+// One CTA per (b, kvh) segment: combine the partials of the pieces that covered it
+// by their log-sum-exps.  Pieces w_first .. w_last of the concatenated key range
+// overlap the segment (none is empty, see effective_pieces); their maxima are
+// reduced first, then their weights exp2(m_w - M) are staged in shared memory a
+// chunk at a time and every thread accumulates its output elements over them.
 template <int D>
 __global__ void __launch_bounds__(128) swa_decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kChunk = 16;           // pieces staged at a time: kChunk x 8 heads = 128 threads
   const int seg = blockIdx.x;
   const int b = seg / a.Hkv, kvh = seg % a.Hkv;
   const int G = a.G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ long long s_red[128];
   __shared__ long long s_info[2];
+  __shared__ float s_wmax[4][8];
+  __shared__ float s_M[8];
+  __shared__ float s_e[kChunk][8];
+  __shared__ float s_el[kChunk][8];
   // Offset of this segment in the concatenated key range, and the total.
   long long before = 0, total = 0;
-  for (int i = threadIdx.x; i < a.B; i += blockDim.x) {
+  for (int i = tid; i < a.B; i += blockDim.x) {
     const long long l = seg_len(a.pos[i], a.W, a.S);
     total += l;
     if (i < b) before += l;
   }
   for (int pass = 0; pass < 2; ++pass) {
-    s_red[threadIdx.x] = pass == 0 ? before : total;
+    s_red[tid] = pass == 0 ? before : total;
     __syncthreads();
     for (int sft = 64; sft > 0; sft >>= 1) {
-      if (threadIdx.x < sft) s_red[threadIdx.x] += s_red[threadIdx.x + sft];
+      if (tid < sft) s_red[tid] += s_red[tid + sft];
       __syncthreads();
     }
-    if (threadIdx.x == 0) s_info[pass] = s_red[0];
+    if (tid == 0) s_info[pass] = s_red[0];
     __syncthreads();
   }
   const long long len = seg_len(a.pos[b], a.W, a.S);
   const long long off = s_info[0] * a.Hkv + kvh * len;
   const long long K = s_info[1] * a.Hkv;
-  const long long Wn = a.n_warps;
-  const long long w_first = ((off + 1) * Wn - 1) / K;
-  const long long w_last = ((off + len) * Wn - 1) / K;
+  const long long Wn = effective_pieces(K, a.n_warps);
+  const long long w_first = ((off + 1) * Wn - 1) / K;   // piece holding key off
+  const long long w_last = ((off + len) * Wn - 1) / K;  // piece holding key off + len - 1
+  const int np = static_cast<int>(w_last - w_first + 1);
   const size_t part_floats = static_cast<size_t>(G) * (D + 2);
+  const float* part0 = a.part + (static_cast<size_t>(w_first) + seg) * part_floats;
 
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int h = idx / D, dim = idx % D;
-    float M = -INFINITY;
-    for (long long w = w_first; w <= w_last; ++w) {
-      if (w * K / Wn == (w + 1) * K / Wn) continue;  // empty piece
-      const float* part = a.part + (static_cast<size_t>(w) + seg) * part_floats;
-      M = fmaxf(M, part[G * D + h]);
+  // 1. the reference max of each head over the pieces
+  float mloc[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) mloc[h] = -INFINITY;
+  for (int p = tid; p < np; p += blockDim.x)
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < G) mloc[h] = fmaxf(mloc[h], part0[p * part_floats + G * D + h]);
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], o));
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int h = 0; h < 8; ++h) s_wmax[warp][h] = mloc[h];
+  __syncthreads();
+  if (tid < 8) s_M[tid] = fmaxf(fmaxf(s_wmax[0][tid], s_wmax[1][tid]), fmaxf(s_wmax[2][tid], s_wmax[3][tid]));
+  __syncthreads();
+
+  // 2. weighted sums, kChunk pieces at a time
+  constexpr int kPer = 8 * D / 128;        // output elements per thread (G <= 8)
+  float acc[kPer], lacc[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) acc[j] = lacc[j] = 0.f;
+  for (int c0 = 0; c0 < np; c0 += kChunk) {
+    {
+      const int p = c0 + tid / 8, h = tid % 8;
+      float e = 0.f, el = 0.f;
+      if (p < np && h < G) {
+        const float* pp = part0 + p * part_floats;
+        e = ex2_approx(pp[G * D + h] - s_M[h]);
+        el = e * pp[G * D + G + h];
+      }
+      s_e[tid / 8][h] = e;
+      s_el[tid / 8][h] = el;
     }
-    float Lsum = 0.f, acc = 0.f;
-    for (long long w = w_first; w <= w_last; ++w) {
-      if (w * K / Wn == (w + 1) * K / Wn) continue;
-      const float* part = a.part + (static_cast<size_t>(w) + seg) * part_floats;
-      const float e = ex2_approx(part[G * D + h] - M);
-      Lsum += e * part[G * D + G + h];
-      acc += e * part[h * D + dim];
+    __syncthreads();
+    const int n = min(kChunk, np - c0);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int idx = tid + 128 * j;
+      if (idx < G * D) {
+        const int h = idx / D, dim = idx % D;
+        const float* pp = part0 + static_cast<size_t>(c0) * part_floats + h * D + dim;
+        for (int p = 0; p < n; ++p) {
+          acc[j] += s_e[p][h] * pp[p * part_floats];
+          lacc[j] += s_el[p][h];
+        }
+      }
     }
-    const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
-    static_cast<__nv_bfloat16*>(a.out)[orow * D + dim] = __float2bfloat16_rn(acc / Lsum);
-    if (dim == 0 && a.lse != nullptr) a.lse[orow] = (M + log2f(Lsum)) * 0.69314718055994531f;
+    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int idx = tid + 128 * j;
+    if (idx < G * D) {
+      const int h = idx / D, dim = idx % D;
+      const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
+      const float o = acc[j] / lacc[j];
+      if (a.out_f32)
+        static_cast<float*>(a.out)[orow * D + dim] = o;
+      else
+        static_cast<__nv_bfloat16*>(a.out)[orow * D + dim] = __float2bfloat16_rn(o);
+      if (dim == 0 && a.lse != nullptr) a.lse[orow] = (s_M[h] + log2f(lacc[j])) * 0.69314718055994531f;
+    }
   }
 }
 

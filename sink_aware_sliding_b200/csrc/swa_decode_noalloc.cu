@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/swa.h"
+#include "swa_internal.h"
 
 namespace {
 
@@ -43,15 +44,16 @@ extern "C" {
 int swa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const void* sink_k,
                        const void* sink_v, const int32_t* pos, void* out, float* lse, int B, int Hq,
                        int Hkv, int d, int window, int n_sink, float scale, swa_stream_t stream) {
+  // swa_decode's own argument checks first, so that an error does not depend on the size.
+  int st = swa::decode_args_status(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window,
+                                   n_sink, scale, SWA_DTYPE_BF16);
+  if (st != SWA_OK) return st;
+  if (B == 0) return SWA_OK;
   const size_t need = swa_decode_workspace_bytes(B, Hq, Hkv, d, window, n_sink);
-  if (need == 0) {
-    // Invalid or unsupported sizes: let swa_decode report which (it launches nothing).
-    return swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window,
-                      n_sink, scale, nullptr, 0, stream);
-  }
+  if (need == 0) return SWA_ERR_CUDA;                    // the device could not be queried
   if (need > kScratchBytes) return SWA_ERR_UNSUPPORTED;  // the fixed scratch is too small
   void* scratch = nullptr;
-  int st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != SWA_OK) return st;
   return swa_decode(q, kcache, vcache, sink_k, sink_v, pos, out, lse, B, Hq, Hkv, d, window, n_sink,
                     scale, scratch, kScratchBytes, stream);

@@ -68,12 +68,13 @@ struct DecodeArgs {
   const void* sink_k;   // [B, Hkv, S, d]
   const void* sink_v;
   const int32_t* pos;   // [B]
-  void* out;            // [B, Hq, d]
+  void* out;            // [B, Hq, d], bf16 or (out_f32) float32
   float* lse;           // [B, Hq] or null
   float* part;          // partial states, (n_warps + B*Hkv) slots
   int B, Hq, Hkv, G, W, S;
   float scale_log2;
   int n_warps;          // total warps of the split kernel
+  int out_f32;          // 1: out is float32
 };
 
 // Rotary frequencies theta_i = base^(-2i/d), i < d/2 (d <= 128), for the fused
@@ -87,6 +88,11 @@ void make_rope_table(double base, int d, RopeTable* t);
 cudaError_t launch_decode(const DecodeArgs& a, int d, int grid, int block, cudaStream_t stream,
                           const RopeTable* rope = nullptr);
 size_t decode_partial_floats(int G, int d);
+// Every argument check of swa_decode_ex except the workspace (SWA_OK when the
+// arguments are valid; B == 0 is valid and means nothing to launch).
+int decode_args_status(const void* q, const void* kcache, const void* vcache, const void* sink_k,
+                       const void* sink_v, const int32_t* pos, const void* out, const float* lse, int B,
+                       int Hq, int Hkv, int d, int window, int n_sink, float scale, int out_dtype);
 cudaError_t decode_occupancy(int d, int B, int* ctas_per_sm);
 int decode_threads();
 

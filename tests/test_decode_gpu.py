@@ -158,3 +158,55 @@ def test_decode_workload_sampled():
                                        w.scale)
             assert_close(out[b:b + 1], ro, f"step {i} b {b} out")
             assert_close(lse[b:b + 1], rl, f"step {i} b {b} lse")
+
+
+def _decode_workload_check(name, steps, rows, out_dtype):
+    w = WORKLOADS[name]
+    di = workloads.make_decode(w, device="cuda", steps=steps)
+    c = Cache(w.B, w.Hkv, w.d, w.window, w.n_sink)
+    c.fill(di.prefix_k, di.prefix_v)
+    nbytes = swa.swa_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.window, w.n_sink)
+    ws = torch.empty(nbytes, device="cuda", dtype=torch.uint8)
+    for i in range(steps):
+        p = w.prefix + i
+        pos = torch.full((w.B,), p, dtype=torch.int32, device="cuda")
+        c.append(di.k_new[i], di.v_new[i], pos)
+        out = torch.empty(w.B, w.Hq, w.d, device="cuda", dtype=out_dtype)
+        lse = torch.empty(w.B, w.Hq, device="cuda", dtype=torch.float32)
+        swa.swa_decode(di.q[i], c.kc, c.vc, c.sk, c.sv, pos, out, lse, w.window, w.n_sink, ws)
+        torch.cuda.synchronize()
+        for b in rows:
+            kh = torch.cat([di.prefix_k[b], di.k_new[:i + 1, b]], 0)[None].cpu()
+            vh = torch.cat([di.prefix_v[b], di.v_new[:i + 1, b]], 0)[None].cpu()
+            ro, rl = oracle.swa_decode(di.q[i, b:b + 1].cpu(), kh, vh, [p], w.window, w.n_sink, w.scale)
+            assert_close(out[b:b + 1], ro, f"{name} step {i} b {b} out")
+            assert_close(lse[b:b + 1], rl, f"{name} step {i} b {b} lse")
+
+
+def test_decode_workload_sampled_f32_output_strict_bound():
+    """The decode workload with a float32 output: the kernels' arithmetic is held to
+    max-abs 1e-2 and mean-abs 1e-3 with no allowance for a final bf16 rounding."""
+    _decode_workload_check("decode", 2, (0, 21, 63), torch.float32)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_decode_single_sequence_workload(out_dtype):
+    """One sequence (B=1, Hq=32, Hkv=8, d=128, window 4096 + 4 sinks) after a 16384-token
+    prefix: the split grid is sized by the visible keys, not the GPU."""
+    _decode_workload_check("decode_b1", 3, (0,), out_dtype)
+
+
+def test_decode_early_positions_few_keys():
+    """Positions 0..5 of a single sequence: far fewer keys than warps in the grid, so
+    most warps take no piece and every piece still holds a key."""
+    B, Hq, Hkv, d, W, S = 1, 32, 8, 128, 4096, 4
+    n = 6
+    k, v, q = rand((B, n, Hkv, d), 17), rand((B, n, Hkv, d), 18), rand((B, n, Hq, d), 19)
+    c = Cache(B, Hkv, d, W, S)
+    for p in range(n):
+        pos = torch.full((B,), p, dtype=torch.int32, device="cuda")
+        c.append(k[:, p], v[:, p], pos)
+        out, lse = decode(c, q[:, p], pos, Hkv)
+        ro, rl = oracle.swa_decode(q[:, p], k, v, [p], W, S, 1 / math.sqrt(d))
+        assert_close(out, ro, f"pos {p} out")
+        assert_close(lse, rl, f"pos {p} lse")

@@ -2,7 +2,13 @@
 memory (their host framework owns every allocation, or allocation is forbidden
 after start-up).  It must give the same results as swa_decode, which takes its
 scratch from the caller, on two calls in a row that share the library's fixed
-scratch array.  This file is collected last on purpose."""
+scratch array.
+
+The file name sorts last so that pytest collects it after every other test file:
+a run that stops at the first failure has then run everything else first, and the
+array is exercised after the other tests have used the library on the same
+device.  Nothing here depends on what the other tests did: the cases also pass in
+a fresh process."""
 import ctypes
 import math
 
@@ -54,11 +60,43 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
         assert_close(lse, rl, f"call {call} lse vs oracle")
 
 
+def test_noalloc_larger_then_smaller_batch_d64_no_sinks_no_lse():
+    """A call with more sequences leaves partial states in the shared array beyond
+    what the next, smaller call writes; the smaller call (d = 64, no sinks, no lse)
+    must not read them."""
+    Hq, Hkv, d, W, S = 4, 2, 64, 48, 0
+    for B, pos, seed in ((7, [0, 9, 47, 48, 60, 130, 200], 3), (2, [5, 100], 4)):
+        k, v, (kc, vc, sk, sv) = _setup(B, Hq, Hkv, d, W, S, pos, seed=seed)
+        pos_d = torch.tensor(pos, dtype=torch.int32, device="cuda")
+        ws = torch.empty(swa.swa_decode_workspace_bytes(B, Hq, Hkv, d, W, S), dtype=torch.uint8, device="cuda")
+        q = torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(20 + B)).bfloat16().cuda()
+        ref = torch.empty(B, Hq, d, device="cuda", dtype=torch.bfloat16)
+        swa.swa_decode(q, kc, vc, sk, sv, pos_d, ref, None, W, S, ws)
+        out = torch.empty_like(ref)
+        swa.swa_decode_noalloc(q, kc, vc, sk, sv, pos_d, out, None, W, S)
+        torch.cuda.synchronize()
+        assert_close(out, ref.double(), f"B={B} out vs swa_decode")
+        ro, _ = oracle.swa_decode(q, k, v, pos, W, S, 1 / math.sqrt(d))
+        assert_close(out, ro, f"B={B} out vs oracle")
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # 4096 sequences x 8 KV heads need far more than the fixed 8 MiB of scratch.
-    lib = swa.library()
-    need = lib.swa_decode_workspace_bytes(4096, 32, 8, 128, 4096, 4)
+    # 4096 sequences x 8 KV heads need far more than the fixed 8 MiB of scratch; the
+    # arguments are otherwise valid, so the size is what is rejected.
+    B, Hq, Hkv, d, W, S = 4096, 32, 8, 128, 4096, 4
+    need = swa.swa_decode_workspace_bytes(B, Hq, Hkv, d, W, S)
     assert need > 8 << 20
-    st = lib.swa_decode_noalloc(None, None, None, None, None, None, None, None, 4096, 32, 8, 128, 4096, 4,
+    z = dict(device="cuda", dtype=torch.bfloat16)
+    q = torch.zeros(B, Hq, d, **z)
+    kc = torch.zeros(B, Hkv, 16, d, **z)          # only pointers are checked before the size
+    sk = torch.zeros(B, Hkv, S, d, **z)
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    with pytest.raises(swa.SwaError) as e:
+        swa.swa_decode_noalloc(q, kc, kc, sk, sk, pos, out, None, W, S)
+    assert e.value.status == swa.SWA_ERR_UNSUPPORTED
+    # invalid arguments are reported as such whatever the size
+    lib = swa.library()
+    st = lib.swa_decode_noalloc(None, None, None, None, None, None, None, None, B, Hq, Hkv, d, W, S,
                                 ctypes.c_float(0.1), None)
-    assert st == swa.SWA_ERR_UNSUPPORTED
+    assert st == swa.SWA_ERR_INVALID_ARG

@@ -93,6 +93,10 @@ WORKLOADS = {
         "decode_rope", "decode", Hq=32, Hkv=8, d=128, window=4096, n_sink=4, dtype="bf16",
         B=64, prefix=16384, steps=1024, sink_bias=True, rope_base=10000.0,
         note="the decode workload with the rotary encoding fused into append and decode"),
+    "decode_b1": Workload(
+        "decode_b1", "decode", Hq=32, Hkv=8, d=128, window=4096, n_sink=4, dtype="bf16",
+        B=1, prefix=16384, steps=1024, sink_bias=True,
+        note="the decode workload for a single sequence (latency-bound serving case)"),
     "packed_long": Workload(
         "packed_long", "varlen", Hq=32, Hkv=8, d=128, window=2048, n_sink=4, dtype="bf16",
         seqlens=(131072, 65536, 16384, 1000), note="four packed sequences"),
