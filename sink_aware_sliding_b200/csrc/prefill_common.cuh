@@ -125,26 +125,26 @@ __device__ __forceinline__ void build_varlen_tables(const PrefillArgs& a, int* s
 // writes P over S (packed bf16 pairs, or fp32 for the tf32 path) and updates
 // the running max and sum.  Returns whether the reference max moved; alpha is
 // the factor the row's O accumulator must be scaled by in that case.
+// Bits [a, b] (inclusive, clipped to the word) of the 32-column word starting at column base.
+__device__ __forceinline__ uint32_t range_bits(int a, int b, int base) {
+  const int lo = max(a - base, 0), hi = min(b - base, 31);
+  if (lo > hi) return 0u;
+  return (0xFFFFFFFFu >> (31 - hi)) & (0xFFFFFFFFu << lo);
+}
+
 // Set the columns of s this row cannot see to -inf.  Visible: c <= hi and
-// (c >= lo or c < sk), all relative to the tile's first key.  The common edge
-// tiles need one compare per element: the diagonal tile (window start left of
-// the tile for every row of the warp) only the causal bound, the lower band
-// edge (tile end at or before every row's position) only the window bound; the
-// general predicate is left for tiles that touch the sink prefix.
+// (c >= lo or c < sk), all relative to the tile's first key.  The visible columns
+// are first gathered into four 32-bit words (two ranges per word), then every
+// column is kept or cleared by its bit: one code path of two instructions per
+// column for every kind of edge tile (diagonal, lower band edge, sink prefix).
 __device__ __forceinline__ void mask_tile(float* s, int hi, int lo, int sk) {
-  const bool no_lo = __all_sync(0xffffffffu, lo <= 0 || sk >= kBN);
-  const bool no_hi = __all_sync(0xffffffffu, hi >= kBN - 1);
-  const bool no_sink = __all_sync(0xffffffffu, sk <= 0);
-  if (no_lo) {
+  uint32_t w[kBN / 32];
 #pragma unroll
-    for (int c = 0; c < kBN; ++c) s[c] = (c <= hi) ? s[c] : -INFINITY;
-  } else if (no_hi && no_sink) {
+  for (int k = 0; k < kBN / 32; ++k)
+    w[k] = range_bits(max(lo, 0), hi, 32 * k) | range_bits(0, min(sk, hi + 1) - 1, 32 * k);
 #pragma unroll
-    for (int c = 0; c < kBN; ++c) s[c] = (c >= lo) ? s[c] : -INFINITY;
-  } else {
-#pragma unroll
-    for (int c = 0; c < kBN; ++c) s[c] = ((c <= hi) && (c >= lo || c < sk)) ? s[c] : -INFINITY;
-  }
+  for (int c = 0; c < kBN; ++c)
+    s[c] = (static_cast<int>(w[c >> 5] << (31 - (c & 31))) < 0) ? s[c] : -INFINITY;
 }
 
 // Online softmax of one key tile for the row this thread owns (TMEM lane).
@@ -313,6 +313,27 @@ __device__ __forceinline__ void stage_row_bf16_d64(uint32_t o_tmem, uint8_t* til
                                     : (static_cast<size_t>(x.seq) * a.Hq + h) * a.L + t;
     a.lse[idx] = lse;
   }
+}
+
+// Descriptor arithmetic for the MMA issue loops.  The start-address field of a
+// shared-memory descriptor holds (address >> 4) in its low 14 bits, and every
+// shared address here lies below 2^18, so adding (bytes >> 4) to a descriptor moves
+// its start by `bytes` without touching the other fields.  The issue loops build
+// one descriptor per tile and step through it with compile-time offsets (in a
+// one-CTA microbenchmark on a B200, tcgen05.mma instructions whose descriptors
+// needed run-time address arithmetic issued at about 90 cycles each, against the
+// tensor pipe's 52 with base + constant).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+// Offset of K-major k-step kk (32 bytes) in a tile of `rows` rows stored as 128-byte
+// column chunks (STEPS_PER_CHUNK k-steps per chunk).
+template <int STEPS_PER_CHUNK, int ROWS>
+__host__ __device__ constexpr uint32_t kmajor_off(int kk) {
+  return static_cast<uint32_t>((kk / STEPS_PER_CHUNK) * (ROWS * 128) + (kk % STEPS_PER_CHUNK) * 32);
+}
+// Offset of MN-major k-step kk of KSTEP rows (128 bytes per row).
+template <int KSTEP>
+__host__ __device__ constexpr uint32_t mnmajor_off(int kk) {
+  return static_cast<uint32_t>(kk * KSTEP * 128);
 }
 
 // Shared-memory matrix descriptors of the operands (see the kernels for the layouts).

@@ -9,13 +9,15 @@
 // Roles (384 threads):
 //   warps 0-3   softmax of tile A (thread r = query row r = TMEM lane r)
 //   warps 4-7   softmax of tile B
-//   warp 8      TMA: the two Q tiles of a unit, then per key tile its K and V
-//               tiles, each into the next slot of one ring of tile-sized slots
+//   warp 8      TMA: the two Q tiles of a unit, then the K and V tiles, K one key
+//               tile ahead of V, each into the next slot of one ring of tile-sized slots
 //   warp 9      tcgen05.mma issue (one thread) and TMEM allocation
 // The MMA order per key tile j is
 //   O_A += P_A(j) V(j);  S_A = Q_A K(j+1)^T;  O_B += P_B(j) V(j);  S_B = Q_B K(j+1)^T
 // so the tensor pipe works on one tile's products while the softmax warps of the
-// other tile run.  Each tile has a single S region in TMEM (P overwrites S in
+// other tile run, and the two tiles' softmax phases stay half a period apart (with
+// one issuer per tile they fell into step and shared the MUFU, 20% slower on a
+// B200).  Each tile has a single S region in TMEM (P overwrites S in
 // place); because the MMAs of one CTA execute in issue order, S_X(j+1) being
 // ready implies O_X += P_X(j) V(j) has finished, so a softmax warp may rescale
 // its O rows right after reading S without a further barrier.
@@ -172,14 +174,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             tma_load_3d(base + C::OFF_Q + (qb * 2 + half) * C::TILE + c * (kBM * 128), &tq,
                         bar(C::B_QFULL + qb), c * C::CHUNK, hA + half, x.seq_start + x.m0);
         last_q[qb] = uc;
-        for (int j = 0; ok && j < x.n_tiles; ++j) {
+        // K runs one key tile ahead of V: K(0), then per tile j K(j+1) and V(j), so that
+        // the K tile a Q K^T needs next is requested a whole tile earlier than its V.
+        // Each group is one slot (the two heads share a KV head) or two (A, then B).
+        const int gsz = shared ? 1 : 2;
+        for (int step = 0; ok && step < 2 * x.n_tiles; ++step) {
+          const bool is_v = step > 0 && (step % 2 == 0 || step == 2 * x.n_tiles - 1);
+          const int j = is_v ? (step == 2 * x.n_tiles - 1 ? x.n_tiles - 1 : step / 2 - 1) : (step + 1) / 2;
           const int row = x.seq_start + tile_n0(x, j);
-          // slots: K_A, [K_B], V_A, [V_B]
-          for (int part = 0; part < (shared ? 2 : 4); ++part, ++ld) {
+          for (int part = 0; part < gsz; ++part, ++ld) {
             const int st = ld % C::NSTAGE;
             if (!(ok = wait_bar(bar(C::B_EMPTY + st), ((ld / C::NSTAGE) & 1) ^ 1, ctl))) break;
-            const bool is_v = shared ? part == 1 : part >= 2;
-            const int kvh = shared ? kvA : ((part & 1) ? kvB : kvA);
+            const int kvh = part ? kvB : kvA;
             mbar_expect_tx(bar(C::B_FULL + st), C::TILE);
             for (int c = 0; c < C::NCHUNK; ++c)
               tma_load_3d(base + C::OFF_RING + st * C::TILE + c * (kBN * 128), is_v ? &tv : &tk,
@@ -205,23 +211,25 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       auto wait_full = [&](int slot_ctr) -> bool {
         return wait_bar(bar(C::B_FULL + slot_ctr % C::NSTAGE), (slot_ctr / C::NSTAGE) & 1, ctl);
       };
-      auto slot_addr = [&](int slot_ctr) -> uint32_t {
-        return base + C::OFF_RING + (slot_ctr % C::NSTAGE) * C::TILE;
-      };
-      auto qk = [&](int half, uint32_t q_tile, int k_ctr) {
-        const uint32_t k_tile = slot_addr(k_ctr);
+      // descriptors of the first Q tile and of ring slot 0; tiles and k-steps are constant offsets
+      constexpr int SPC = C::QK_STEPS / C::NCHUNK;
+      const uint64_t dq0 = kmajor_desc<SPC>(base + C::OFF_Q, kBM, 0);
+      const uint64_t dk0 = kmajor_desc<SPC>(base + C::OFF_RING, kBN, 0);
+      const uint64_t dv0 = v_desc<F32, C::KSTEP>(base + C::OFF_RING, 0);
+      auto qk = [&](int half, uint64_t dq, int k_ctr) {
+        const uint64_t dk = desc_add(dk0, (k_ctr % C::NSTAGE) * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<F32>(tmem + C::tmem_s(half), kmajor_desc<C::QK_STEPS / C::NCHUNK>(q_tile, kBM, kk),
-                       kmajor_desc<C::QK_STEPS / C::NCHUNK>(k_tile, kBN, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_ss<F32>(tmem + C::tmem_s(half), desc_add(dq, kmajor_off<SPC, kBM>(kk)),
+                       desc_add(dk, kmajor_off<SPC, kBN>(kk)), C::IDESC_QK, kk > 0 ? 1u : 0u);
         tc_commit(bar(C::B_SFULL + half));
       };
       auto pv = [&](int half, int v_ctr, bool first) {
-        const uint32_t v_tile = slot_addr(v_ctr);
+        const uint64_t dv = desc_add(dv0, (v_ctr % C::NSTAGE) * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<F32>(tmem + C::tmem_o(half), tmem + C::tmem_s(half) + kk * 8,
-                       v_desc<F32, C::KSTEP>(v_tile, kk), C::IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          umma_ts<F32>(tmem + C::tmem_o(half), tmem + C::tmem_s(half) + kk * 8, desc_add(dv, mnmajor_off<C::KSTEP>(kk)),
+                       C::IDESC_PV, (first && kk == 0) ? 0u : 1u);
       };
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
         Unit x;
@@ -230,14 +238,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const bool shared = hA / a.G == (hA + 1) / a.G;
         const int per = shared ? 2 : 4;
         const int qb = uc % C::QBUF;
-        const uint32_t qA = base + C::OFF_Q + (qb * 2) * C::TILE, qB = qA + C::TILE;
+        const uint64_t qA = desc_add(dq0, (qb * 2) * C::TILE), qB = desc_add(qA, C::TILE);
         if (!(ok = wait_bar(bar(C::B_QFULL + qb), (uc / C::QBUF) & 1, ctl))) break;
-        // slots of tile j: base b_j = ld + j*per; K_A = b_j, K_B = b_j + (shared ? 0 : 1),
-        // V_A = b_j + (shared ? 1 : 2), V_B = V_A + (shared ? 0 : 1)
-        auto kA = [&](int j) { return ld + j * per; };
-        auto kB = [&](int j) { return ld + j * per + (shared ? 0 : 1); };
-        auto vA = [&](int j) { return ld + j * per + (shared ? 1 : 2); };
-        auto vB = [&](int j) { return ld + j * per + (shared ? 1 : 3); };
+        // ring positions in the load order K(0), K(1), V(0), K(2), V(1), ..., V(n-1), in groups
+        // of g = per / 2 slots (A, then B when the heads read different KV heads)
+        const int g = per / 2, nt = x.n_tiles;
+        auto kA = [&](int j) { return ld + (j == 0 ? 0 : (2 * j - 1) * g); };
+        auto kB = [&](int j) { return kA(j) + (shared ? 0 : 1); };
+        auto vA = [&](int j) { return ld + (j == nt - 1 ? 2 * nt - 1 : 2 * j + 2) * g; };
+        auto vB = [&](int j) { return vA(j) + (shared ? 0 : 1); };
         // prologue: S_A(0), S_B(0)
         if (!(ok = wait_full(kA(0)) && (shared || wait_full(kB(0))))) break;
         tc_fence_after();

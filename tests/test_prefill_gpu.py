@@ -84,6 +84,9 @@ def test_tiny_workload_fp32():
     (1, 900, 6, 2, 64, 256, 4),        # same at d = 64 (two-tile kernel, separate K/V)
     (4, 1024, 16, 16, 64, 128, 0),     # many units per CTA, d = 64, G = 1
     (1, 4096, 32, 8, 128, 512, 4),     # many units per CTA, GQA
+    (1, 500, 4, 2, 128, 40, 4),        # sink tile is the first band tile
+    (1, 500, 4, 2, 64, 40, 70),        # sink prefix across the first band tile, d = 64
+    (2, 640, 4, 2, 64, 200, 4),        # d = 64 GQA: TMA-store epilogue over several units
 ])
 def test_prefill_matches_oracle(B, L, Hq, Hkv, d, window, n_sink):
     q, k, v = rand_qkv(B, L, Hq, Hkv, d, seed=B * 1000 + L)

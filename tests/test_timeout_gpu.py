@@ -22,15 +22,15 @@ def _inputs(Hq, Hkv, d=128, L=512):
     return q, k, v
 
 
-@pytest.mark.parametrize("one_tile", [False, True])
-def test_expired_wait_reports_timeout_and_context_survives(one_tile):
+@pytest.mark.parametrize("kernel_flags", [0, 2], ids=["two-tile", "one-tile"])
+def test_expired_wait_reports_timeout_and_context_survives(kernel_flags):
     q, k, v = _inputs(8, 2)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     out = torch.zeros_like(qd)
     lse = torch.zeros(1, 8, 512, device="cuda")
     assert swa.swa_device_error() == 0
     prev_t = swa.swa_set_wait_timeout_ns(50_000_000)          # 50 ms
-    prev_f = swa.swa_set_debug_flags(1 | (2 if one_tile else 0))
+    prev_f = swa.swa_set_debug_flags(1 | kernel_flags)
     try:
         swa.swa_fwd(qd, kd, vd, out, lse, 128, 4)
         assert swa.swa_device_error() == swa.SWA_ERR_DEVICE_TIMEOUT
