@@ -162,7 +162,7 @@ int run_prefill(const void* q, const void* k, const void* v, void* out, float* l
 // Split-K decode grid: one warp per kDecodeKeysPerWarp keys of the largest
 // possible visible set (every segment holds at most window + n_sink keys; the
 // positions themselves are on the device), and never more CTAs than fill the GPU.
-constexpr long long kDecodeKeysPerWarp = 32;
+constexpr long long kDecodeKeysPerWarp = 64;
 int decode_grid(DeviceInfo* dev, int d, int B, int Hkv, int window, int n_sink, int* grid) {
   const int idx = d == 128 ? 1 : 0;
   if (dev->decode_ctas_per_sm[idx] == 0) {

@@ -18,8 +18,12 @@
 // A third, small kernel computes D_t = rowsum(dO_t O_t) for every row first,
 // into the storage of dq (which the dQ kernel only writes after the dK/dV kernel
 // has read D; the dQ kernel forms its own D per row).
-// Each CTA is one warpgroup; thread 0 issues TMA and MMA, all threads do the
-// element-wise step; every hand-off is an mbarrier with a bounded wait.  Thread 0
+// Each CTA is two warpgroups over the same 128 TMEM lanes: the first does the
+// element-wise step on score columns 0-63, the second on columns 64-127 (the step
+// is independent per column), so each thread handles half a row.  Visibility is
+// tested only on edge tiles, through four 32-bit words per row built from the row's
+// visible column ranges.  Thread 0 issues TMA and MMA; every hand-off is an
+// mbarrier with a bounded wait.  Thread 0
 // shares warp 0 with element-wise threads, so the warp is reconverged
 // (__syncwarp) after every issuer-only block and every wait's outcome is made
 // warp-uniform before the warp-collective tcgen05 instructions that follow.  The
@@ -45,7 +49,8 @@ namespace {
 
 using namespace prefill;
 
-constexpr int kBwdThreads = 128;
+constexpr int kBwdThreads = 256;
+constexpr int kRowThreads = 128;   // the first warpgroup also stages the per-row data
 
 template <int D>
 struct BwdCfg {
@@ -112,8 +117,14 @@ __device__ __forceinline__ float row_dot(const __nv_bfloat16* x, const __nv_bflo
   return acc;
 }
 
-__device__ __forceinline__ bool visible(int j, int t, const PrefillArgs& a) {
-  return j <= t && t < a.L && (j >= t - a.window + 1 || j < a.n_sink);
+// Columns c in [0, 128) of a score tile whose absolute index lies in [lo, hi] or in
+// [0, sk_hi], as four 32-bit words (bit c of word c / 32).
+__device__ __forceinline__ void visible_words(int lo, int hi, int sk_hi, uint32_t* w) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w[k] = range_bits(lo, hi, 32 * k) | range_bits(0, sk_hi, 32 * k);
+}
+__device__ __forceinline__ bool word_bit(const uint32_t* w, int c) {
+  return static_cast<int>(w[c >> 5] << (31 - (c & 31))) < 0;
 }
 
 template <int D>
@@ -166,7 +177,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                   : min(tiles - 1, (min(j0 + kBN - 1, a.L - 1) + a.window - 1) / kBM);
 
   if (tid == 0) {
-    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), (i == kBarP || i == kBarRow) ? kBwdThreads : 1);
+    for (int i = 0; i < C::NBAR; ++i)
+      mbar_init(bar(i), i == kBarP ? kBwdThreads : (i == kBarRow ? kRowThreads : 1));
     fence_mbar_init();
   }
   __syncwarp();
@@ -178,7 +190,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const uint32_t lane_off = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+  const int r = tid & 127;                            // TMEM lane (key row) of this thread
+  const int half = tid >> 7;                          // score columns 64 half .. 64 half + 63
+  const bool stager = tid < kRowThreads;
+  const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
   const size_t row_base = static_cast<size_t>(b) * a.L;
 
   // iterations: (query head g, query tile) flattened, query tiles fastest
@@ -193,8 +208,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     load_tile<D>(sdO + 2 * buf * C::TILE, &tdo, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
   };
   const float* d_rows = ba.dq;                        // D, written by the D kernel
-  auto fetch_row = [&](int i, float& dt, float& l2) { // D and lse (log2 units) of query it_row0(i) + tid
-    const int t = it_row0(i) + tid;
+  auto fetch_row = [&](int i, float& dt, float& l2) { // D and lse (log2 units) of query it_row0(i) + r
+    const int t = it_row0(i) + r;
     const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + t;
     dt = t < a.L ? d_rows[idx] : 0.f;
     l2 = t < a.L ? ba.lse[idx] * 1.4426950408889634f : 0.f;
@@ -204,10 +219,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // into registers would wait for them to land.
   const uint32_t stg = smem_u32(gbase + C::OFF_STG);
   auto stage_row = [&](int i) {
-    const int t = it_row0(i) + tid;
+    const int t = it_row0(i) + r;
     const bool in = t < a.L;
     const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + (in ? t : 0);
-    const uint32_t dst = stg + (i & 1) * 1024 + tid * 4;
+    const uint32_t dst = stg + (i & 1) * 1024 + r * 4;
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(d_rows + idx), "r"(in ? 4u : 0u)
                  : "memory");
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 512), "l"(ba.lse + idx), "r"(in ? 4u : 0u)
@@ -224,12 +239,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     issue(0);
     issued = 1;
   }
-  float next_d = 0.f, next_l = 0.f;
-  fetch_row(0, next_d, next_l);
-  D_s[tid] = next_d;
-  L_s[tid] = next_l;
-  mbar_arrive(bar(kBarRow));
-  const int s_key = j0 + tid;                         // this thread's key (TMEM lane)
+  if (stager) {
+    float next_d = 0.f, next_l = 0.f;
+    fetch_row(0, next_d, next_l);
+    D_s[r] = next_d;
+    L_s[r] = next_l;
+    mbar_arrive(bar(kBarRow));
+  }
+  const int s_key = j0 + r;                           // this thread's key (TMEM lane)
+  // query rows that see this key: s_key .. s_key + window - 1 (all later rows for a
+  // sink), before the sequence's end
+  const int t_hi = min(a.L - 1, s_key < a.n_sink ? a.L - 1 : s_key + a.window - 1);
   int it = 0;
   for (; it < n_it; ++it) {
     const int i0 = it_row0(it), buf = it & 1;
@@ -240,7 +260,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       issue(it + 1);
       issued = it + 2;
     }
-    if (it + 1 < n_it) stage_row(it + 1);
+    if (stager && it + 1 < n_it) stage_row(it + 1);
     __syncwarp();
     if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
     if (tid == 0) {
@@ -261,14 +281,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), it & 1, a)))) break;
     tc_fence_after();
-    // P^T and dS^T of this key row, 64 query columns at a time
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
+    // P^T and dS^T of this key row over this warpgroup's 64 query columns
+    {
+      // every (key, query) pair of the tile visible: no test per column
+      const bool full = j0 + kBN - 1 <= i0 && i0 + kBM - 1 < a.L &&
+                        (j0 >= i0 + kBM - a.window || j0 + kBN - 1 < a.n_sink);
+      uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
+      if (!full) visible_words(s_key - i0, t_hi - i0, -1, vw);
       uint32_t sr[64], dr[64];
-      tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
-      tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
-      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
-      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
+      tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
+      tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
       uint32_t pw[32], dw[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
@@ -276,8 +298,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int col = 64 * half + c + e;
-          const bool vis = visible(s_key, i0 + col, a);
-          p[e] = vis ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]) : 0.f;
+          const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]);
+          p[e] = word_bit(vw, col) ? pe : 0.f;
           ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
         }
         pw[c / 2] = pack_bf16x2(p[0], p[1]);
@@ -306,11 +328,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
     // every thread is past this iteration's element-wise step: publish the next row data
-    if (it + 1 < n_it) {
+    if (stager && it + 1 < n_it) {
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       const float* st = reinterpret_cast<const float*>(gbase + C::OFF_STG + ((it + 1) & 1) * 1024);
-      D_s[tid] = st[tid];
-      L_s[tid] = st[128 + tid] * 1.4426950408889634f;
+      D_s[r] = st[r];
+      L_s[r] = st[128 + r] * 1.4426950408889634f;
       mbar_arrive(bar(kBarRow));
     }
   }
@@ -328,7 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* dv = ba.dv + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
     float* dk = ba.dk + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
       uint32_t rv[32], rk[32];
       tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, rv);
       tmem_ld32_wait(tmem + lane_off + 256 + D + 32 * c, rk);
@@ -387,9 +409,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const uint32_t lane_off = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+  const int r = tid & 127;                            // TMEM lane (query row) of this thread
+  const int half = tid >> 7;                          // key columns 64 half .. 64 half + 63
+  const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
   const size_t row_base = static_cast<size_t>(b) * a.L;
-  const int t = x.m0 + tid;                           // this thread's query row
+  const int t = x.m0 + r;                             // this thread's query row
 
   bool ok = true;
   int issued = 0;                                     // key tiles whose K, V were requested
@@ -439,22 +463,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
     if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), j & 1, a)))) break;
     tc_fence_after();
-    // dS of this query row, 64 key columns at a time, written over S
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
+    // dS of this query row over this warpgroup's 64 key columns, written over S
+    {
+      uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
+      if (tile_needs_mask(x, j, a.window) || x.m1 - x.m0 != kBM - 1) {
+        // keys t - window + 1 .. t and the sinks below min(n_sink, t + 1); nothing past the end
+        if (t < a.L) visible_words(t - a.window + 1 - n0, t - n0, min(a.n_sink, t + 1) - 1 - n0, vw);
+        else vw[0] = vw[1] = vw[2] = vw[3] = 0u;
+      }
       uint32_t sr[64], dr[64];
-      tmem_ld32_wait(tmem + lane_off + 64 * half, sr);
-      tmem_ld32_wait(tmem + lane_off + 64 * half + 32, sr + 32);
-      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half, dr);
-      tmem_ld32_wait(tmem + lane_off + 128 + 64 * half + 32, dr + 32);
+      tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
+      tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
       uint32_t dw[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         float ds[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int key = n0 + 64 * half + c + e;
-          const float p = visible(key, t, a) ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - l2) : 0.f;
+          const int col = 64 * half + c + e;
+          const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - l2);
+          const float p = word_bit(vw, col) ? pe : 0.f;
           ds[e] = p * (__uint_as_float(dr[c + e]) - dt);
         }
         dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
@@ -489,7 +517,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool row_ok = t < a.L;
     float* dq = ba.dq + ((row_base + (row_ok ? t : 0)) * a.Hq + h) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
       uint32_t r[32];
       tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, r);
       if (!row_ok) continue;

@@ -297,44 +297,51 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 }
 
-// One CTA per (b, kvh) segment: combine the partials of the pieces that covered it
-// by their log-sum-exps.  Pieces w_first .. w_last of the concatenated key range
-// overlap the segment (none is empty, see effective_pieces); their maxima are
-// reduced first, then their weights exp2(m_w - M) are staged in shared memory a
-// chunk at a time and every thread accumulates its output elements over them.
+// One CTA per (b, kvh) segment and query head h of that KV head, D threads (one output
+// element each): combine the partials of the pieces that covered the segment by their
+// log-sum-exps.  Pieces w_first .. w_last of the concatenated key range overlap the
+// segment (none is empty, see effective_pieces).  The head's maximum over the pieces
+// is reduced first; then the weights exp2(m_w - M) are staged in shared memory a chunk
+// at a time and every thread accumulates its element over them, with the loads of a
+// chunk in flight together.
 template <int D>
-__global__ void __launch_bounds__(128) swa_decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int kChunk = 16;           // pieces staged at a time: kChunk x 8 heads = 128 threads
+__global__ void __launch_bounds__(D) swa_decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kChunk = D;
   const int seg = blockIdx.x;
+  const int h = blockIdx.y;
   const int b = seg / a.Hkv, kvh = seg % a.Hkv;
   const int G = a.G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ long long s_red[128];
-  __shared__ long long s_info[2];
-  __shared__ float s_wmax[4][8];
-  __shared__ float s_M[8];
-  __shared__ float s_e[kChunk][8];
-  __shared__ float s_el[kChunk][8];
+  __shared__ long long s_red[D / 32][2];
+  __shared__ float s_wmax[D / 32];
+  __shared__ float s_e[kChunk];
+  __shared__ float s_el[kChunk];
   // Offset of this segment in the concatenated key range, and the total.
   long long before = 0, total = 0;
-  for (int i = tid; i < a.B; i += blockDim.x) {
+  for (int i = tid; i < a.B; i += D) {
     const long long l = seg_len(a.pos[i], a.W, a.S);
     total += l;
     if (i < b) before += l;
   }
-  for (int pass = 0; pass < 2; ++pass) {
-    s_red[tid] = pass == 0 ? before : total;
-    __syncthreads();
-    for (int sft = 64; sft > 0; sft >>= 1) {
-      if (tid < sft) s_red[tid] += s_red[tid + sft];
-      __syncthreads();
-    }
-    if (tid == 0) s_info[pass] = s_red[0];
-    __syncthreads();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  if (lane == 0) {
+    s_red[warp][0] = before;
+    s_red[warp][1] = total;
+  }
+  __syncthreads();
+  before = total = 0;
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) {
+    before += s_red[w][0];
+    total += s_red[w][1];
   }
   const long long len = seg_len(a.pos[b], a.W, a.S);
-  const long long off = s_info[0] * a.Hkv + kvh * len;
-  const long long K = s_info[1] * a.Hkv;
+  const long long off = before * a.Hkv + kvh * len;
+  const long long K = total * a.Hkv;
   const long long Wn = effective_pieces(K, a.n_warps);
   const long long w_first = ((off + 1) * Wn - 1) / K;   // piece holding key off
   const long long w_last = ((off + len) * Wn - 1) / K;  // piece holding key off + len - 1
@@ -342,73 +349,58 @@ __global__ void __launch_bounds__(128) swa_decode_merge_kernel(const __grid_cons
   const size_t part_floats = static_cast<size_t>(G) * (D + 2);
   const float* part0 = a.part + (static_cast<size_t>(w_first) + seg) * part_floats;
 
-  // 1. the reference max of each head over the pieces
-  float mloc[8];
+  // 1. this head's reference max over the pieces
+  float m = -INFINITY;
+  for (int p = tid; p < np; p += D) m = fmaxf(m, part0[p * part_floats + G * D + h]);
 #pragma unroll
-  for (int h = 0; h < 8; ++h) mloc[h] = -INFINITY;
-  for (int p = tid; p < np; p += blockDim.x)
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-      if (h < G) mloc[h] = fmaxf(mloc[h], part0[p * part_floats + G * D + h]);
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mloc[h] = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], o));
-  }
-  if (lane == 0)
-#pragma unroll
-    for (int h = 0; h < 8; ++h) s_wmax[warp][h] = mloc[h];
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_wmax[warp] = m;
   __syncthreads();
-  if (tid < 8) s_M[tid] = fmaxf(fmaxf(s_wmax[0][tid], s_wmax[1][tid]), fmaxf(s_wmax[2][tid], s_wmax[3][tid]));
-  __syncthreads();
+  float M = s_wmax[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_wmax[w]);
 
   // 2. weighted sums, kChunk pieces at a time
-  constexpr int kPer = 8 * D / 128;        // output elements per thread (G <= 8)
-  float acc[kPer], lacc[kPer];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) acc[j] = lacc[j] = 0.f;
+  float acc = 0.f, lacc = 0.f;
   for (int c0 = 0; c0 < np; c0 += kChunk) {
     {
-      const int p = c0 + tid / 8, h = tid % 8;
+      const int p = c0 + tid;
       float e = 0.f, el = 0.f;
-      if (p < np && h < G) {
+      if (p < np) {
         const float* pp = part0 + p * part_floats;
-        e = ex2_approx(pp[G * D + h] - s_M[h]);
+        e = ex2_approx(pp[G * D + h] - M);
         el = e * pp[G * D + G + h];
       }
-      s_e[tid / 8][h] = e;
-      s_el[tid / 8][h] = el;
+      s_e[tid] = e;
+      s_el[tid] = el;
     }
     __syncthreads();
     const int n = min(kChunk, np - c0);
+    const float* pp = part0 + static_cast<size_t>(c0) * part_floats + h * D + tid;
+    int p = 0;
+    for (; p + 8 <= n; p += 8) {
+      float v[8];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int idx = tid + 128 * j;
-      if (idx < G * D) {
-        const int h = idx / D, dim = idx % D;
-        const float* pp = part0 + static_cast<size_t>(c0) * part_floats + h * D + dim;
-        for (int p = 0; p < n; ++p) {
-          acc[j] += s_e[p][h] * pp[p * part_floats];
-          lacc[j] += s_el[p][h];
-        }
+      for (int u = 0; u < 8; ++u) v[u] = pp[(p + u) * part_floats];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc += s_e[p + u] * v[u];
+        lacc += s_el[p + u];
       }
+    }
+    for (; p < n; ++p) {
+      acc += s_e[p] * pp[p * part_floats];
+      lacc += s_el[p];
     }
     __syncthreads();
   }
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int idx = tid + 128 * j;
-    if (idx < G * D) {
-      const int h = idx / D, dim = idx % D;
-      const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
-      const float o = acc[j] / lacc[j];
-      if (a.out_f32)
-        static_cast<float*>(a.out)[orow * D + dim] = o;
-      else
-        static_cast<__nv_bfloat16*>(a.out)[orow * D + dim] = __float2bfloat16_rn(o);
-      if (dim == 0 && a.lse != nullptr) a.lse[orow] = (s_M[h] + log2f(lacc[j])) * 0.69314718055994531f;
-    }
-  }
+  const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
+  const float o = acc / lacc;
+  if (a.out_f32)
+    static_cast<float*>(a.out)[orow * D + tid] = o;
+  else
+    static_cast<__nv_bfloat16*>(a.out)[orow * D + tid] = __float2bfloat16_rn(o);
+  if (tid == 0 && a.lse != nullptr) a.lse[orow] = (M + log2f(lacc)) * 0.69314718055994531f;
 }
 
 template <int D>
@@ -423,7 +415,7 @@ cudaError_t launch_decode_impl(const DecodeArgs& a, int grid, int block, cudaStr
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  swa_decode_merge_kernel<D><<<a.B * a.Hkv, 128, 0, stream>>>(a);
+  swa_decode_merge_kernel<D><<<dim3(a.B * a.Hkv, a.G), D, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -77,3 +77,68 @@ def test_bwd_repeat_is_deterministic():
     _, (a1, b1, c1) = run_bwd(1, 400, 2, 2, 128, 100, 4, 9)
     _, (a2, b2, c2) = run_bwd(1, 400, 2, 2, 128, 100, 4, 9)
     assert torch.equal(a1, a2) and torch.equal(b1, b2) and torch.equal(c1, c2)
+
+
+def test_bwd_gqa_sink_biased_long_sequence():
+    """Near the benchmarked backward shape: four query heads per KV head, d = 128,
+    sink keys biased toward the queries (the 8B-shaped workload's recipe), and a
+    sequence of 32 query tiles, so the dK/dV tile that holds the sink prefix is seen
+    by every later query tile of all four heads."""
+    import workloads
+    B, L, Hq, Hkv, d, window, n_sink = 1, 4096, 8, 2, 128, 1024, 4
+    g = torch.Generator().manual_seed(41)
+    q = torch.randn(B, L, Hq, d, generator=g)
+    k = torch.randn(B, L, Hkv, d, generator=g)
+    v = torch.randn(B, L, Hkv, d, generator=g)
+    do = torch.randn(B, L, Hq, d, generator=g)
+    workloads._bias_sinks_(k[0], q[0], n_sink, Hq // Hkv)
+    q, k, v, do = (t.bfloat16() for t in (q, k, v, do))
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out = torch.empty_like(qd)
+    lse = torch.empty(B, Hq, L, device="cuda")
+    swa.swa_fwd(qd, kd, vd, out, lse, window, n_sink)
+    dq = torch.full((B, L, Hq, d), float("nan"), device="cuda")
+    dk = torch.full((B, L, Hkv, d), float("nan"), device="cuda")
+    dv = torch.full_like(dk, float("nan"))
+    swa.swa_bwd(qd, kd, vd, out, dod, lse, dq, dk, dv, window, n_sink)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    rq, rk, rv = oracle.swa_bwd(q, k, v, do, window, n_sink, 1 / math.sqrt(d))
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk, rk, "dk")
+    assert_grad_close(dv, rv, "dv")
+    # the sink keys carry gradient from every query tile
+    assert np.abs(rk[0, :n_sink]).max() > 0
+
+
+def test_bwd_benchmark_shape_identities():
+    """The benchmarked backward shape itself (B=1, Hq=32, Hkv=8, L=8192, d=128, window
+    4096, 4 sink-biased keys) against two identities that hold at any size: every row
+    of P sums to one, so the dV of a KV head summed over positions equals dout summed
+    over positions and over its query heads; every row of dS sums to zero, so the dK
+    of a KV head sums to zero over positions."""
+    import workloads
+    w = workloads.WORKLOADS["gqa8b_prefill"]
+    q, k, v = workloads.make_prefill(w, device="cuda", L=8192)
+    gen = torch.Generator(device="cuda").manual_seed(workloads.SEED + 1)
+    do = torch.randn(q.shape, generator=gen, device="cuda").bfloat16()
+    out = torch.empty_like(q)
+    lse = torch.empty(1, w.Hq, 8192, device="cuda")
+    swa.swa_fwd(q, k, v, out, lse, w.window, w.n_sink)
+    dq = torch.empty(q.shape, device="cuda")
+    dk = torch.empty(k.shape, device="cuda")
+    dv = torch.empty_like(dk)
+    swa.swa_bwd(q, k, v, out, do, lse, dq, dk, dv, w.window, w.n_sink)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    assert torch.isfinite(dq).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all()
+    G = w.Hq // w.Hkv
+    want_dv = do.double().sum(dim=1).view(1, w.Hkv, G, w.d).sum(dim=2)       # [1, Hkv, d]
+    got_dv = dv.double().sum(dim=1)
+    # P is rounded to bf16 (relative 2^-9 per weight) before P^T dout: the column sums
+    # agree to that relative precision of the summed magnitudes
+    scale_dv = do.double().abs().sum(dim=1).view(1, w.Hkv, G, w.d).sum(dim=2)
+    assert ((got_dv - want_dv).abs() <= 4e-3 * scale_dv + 1e-3).all()
+    got_dk = dk.double().sum(dim=1)
+    scale_dk = dk.double().abs().sum(dim=1)
+    assert ((got_dk.abs()) <= 1e-2 * scale_dk + 1e-3).all()
