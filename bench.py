@@ -663,11 +663,11 @@ def bench_based_linear_decode(name, steps, warmup, dev, flush, peaks, sampler):
 
 
 def bench_hybrid_decode(name, steps, warmup, dev, flush, peaks, sampler):
-    """Decode of a Based-style hybrid layer after a 2048-token prefix: per generated
-    token and sequence, the window branch appends to its 128-slot ring cache and
-    decodes over it (H=16, d=64, no sinks), and the linear branch takes its recurrent
-    step on its fixed-size state (H=16, dk=16, dv=64).  B=64 sequences; the state
-    (72.7 MB) and cache (33.6 MB) fit L2 together, so L2 is flushed before each step."""
+    """Decode of a Based-style hybrid layer after a 2048-token prefix, one launch per
+    generated token (swa_hybrid_decode): the window branch appends to its 128-slot ring
+    cache and decodes over it (H=16, d=64, no sinks), and the linear branch takes its
+    recurrent step on its fixed-size state (H=16, dk=16, dv=64).  B=64 sequences; the
+    state (72.7 MB) and cache (33.6 MB) fit L2 together, so L2 is flushed before each step."""
     import torch
 
     import sink_aware_sliding_b200 as swa
@@ -699,12 +699,10 @@ def bench_hybrid_decode(name, steps, warmup, dev, flush, peaks, sampler):
     out_w = torch.empty(B, H, d, **z16)
     out_l = torch.empty(B, H, lw.dv, **z16)
     lse = torch.empty(B, H, device=dev, dtype=torch.float32)
-    ws = torch.empty(swa.swa_decode_workspace_bytes(B, H, H, d, W, 0), device=dev, dtype=torch.uint8)
 
     def step(i):
-        swa.swa_cache_append(kn[i], vn[i], pos[i], kc, vc, sk, sk, W, 0)
-        swa.swa_decode(q[i], kc, vc, sk, sk, pos[i], out_w, lse, W, 0, ws)
-        swa.swa_based_linear_decode(qd[i], kd[i], vd[i], S, zs, out_l, lw.scale)
+        swa.swa_hybrid_decode(q[i], kn[i], vn[i], pos[i], kc, vc, sk, sk, out_w, lse, W, 0,
+                              qd[i], kd[i], vd[i], S, zs, out_l, scale_l=lw.scale)
 
     for i in range(warmup):
         flush.fill_(1)
@@ -727,15 +725,48 @@ def bench_hybrid_decode(name, steps, warmup, dev, flush, peaks, sampler):
     alg_bytes = (2 * B * H * W * d * 2 + 2 * B * H * d * 2 + 2 * B * H * d * 2 + 8 * B * H
                  + based_linear_decode_bytes(lw, B))
     gbs = alg_bytes / (ms * 1e-3) / 1e9
+
+    # end to end: the step's inputs from pinned host memory, both branches' outputs back
+    host_in = [x[warmup].cpu().pin_memory() for x in (q, kn, vn, qd, kd, vd, pos)]
+    dev_in = [torch.empty_like(x, device=dev) for x in host_in]
+    ho_w = torch.empty(out_w.shape, dtype=out_w.dtype).pin_memory()
+    ho_l = torch.empty(out_l.shape, dtype=out_l.dtype).pin_memory()
+
+    def e2e_step():
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        dq_, dk_, dv_, dql, dkl, dvl, dp = dev_in
+        swa.swa_hybrid_decode(dq_, dk_, dv_, dp, kc, vc, sk, sk, out_w, lse, W, 0, dql, dkl, dvl, S, zs, out_l,
+                              scale_l=lw.scale)
+        ho_w.copy_(out_w, non_blocking=True)
+        ho_l.copy_(out_l, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(dev)
+    n_e2e = max(8, steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / n_e2e
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = ho_w.numel() * ho_w.element_size() + ho_l.numel() * ho_l.element_size()
     roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"], "traffic": None,
-            "algorithmic_bytes_per_launch": alg_bytes}
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+            "traffic": profiled_traffic(name), "algorithmic_bytes_per_launch": alg_bytes}
     return {
         "config": {"workload": name, "kind": "hybrid_decode", "B": B, "H": H, "window": W, "d": d,
                    "linear_dk": lw.dk, "linear_dv": lw.dv, "prefix": P},
         "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5),
         "tokens_per_s": round(B / (ms * 1e-3), 1), "roofline": roof,
-        "e2e": None, "gpu_launches": 4 * steps, "l2": "flushed between steps (512 MiB write)",
+        "e2e": {"value": round(B / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": steps, "l2": "flushed between steps (512 MiB write)",
     }
 
 
@@ -783,7 +814,8 @@ def bench_bwd(name, steps, warmup, dev, flush, peaks, sampler):
     tflops = flops / (ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": round(tflops / peaks["bf16_tflops"], 4), "peak_source": peaks["source"],
-            "flops_per_launch": flops, "traffic": None}
+            "flops_per_launch": flops, "traffic": profiled_traffic(name),
+            "traffic_kernel": "swa_bwd_dkdv_kernel"}
     cfg = dict(w.describe(), L=Lr, workload=name, **{"pass": "backward"})
     return {"config": cfg, "value": round(tflops, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
             "roofline": roof, "gpu_launches": 2 * steps, "l2": "flushed between steps (512 MiB write)"}
@@ -1101,6 +1133,23 @@ def profile_case(args):
         if swa.swa_device_error() != 0:
             raise SystemExit("device wait timed out")
         return
+    if args.profile_case == "hybrid_decode":
+        lw = wl.LINEAR_WORKLOADS["based_linear"]
+        B, H, d, W = args.B or 64, lw.H, 64, 128
+        z16 = dict(device=dev, dtype=torch.bfloat16)
+        kc, vc = torch.randn(B, H, W, d, device=dev).bfloat16(), torch.randn(B, H, W, d, device=dev).bfloat16()
+        S = torch.randn(B, H, lw.F, lw.dv, device=dev)
+        zs = 100.0 + torch.rand(B, H, lw.F, device=dev)
+        q, kn, vn = (torch.randn(B, H, d, device=dev).bfloat16() for _ in range(3))
+        ql, kl = (torch.randn(B, H, lw.dk, device=dev).bfloat16() for _ in range(2))
+        vl = torch.randn(B, H, lw.dv, device=dev).bfloat16()
+        out_w, out_l = torch.empty(B, H, d, **z16), torch.empty(B, H, lw.dv, **z16)
+        for i in range(n):
+            pos = torch.full((B,), 4096 + i, dtype=torch.int32, device=dev)
+            swa.swa_hybrid_decode(q, kn, vn, pos, kc, vc, kc, kc, out_w, None, W, 0, ql, kl, vl, S, zs, out_l,
+                                  scale_l=lw.scale)
+        torch.cuda.synchronize()
+        return
     if args.profile_case in ("based_linear", "based_linear_decode"):
         w = wl.LINEAR_WORKLOADS["based_linear"]
         q, k, v = wl.make_based_linear(w, device=dev, B=args.B, L=args.L)
@@ -1133,7 +1182,8 @@ def profile_case(args):
         for _ in range(n):
             swa.swa_fwd(q, k, v, out, lse, w.window, w.n_sink)
     elif w.kind == "varlen":
-        q, k, v, cu = wl.make_varlen(w, device=dev)
+        seqlens = [int(x) for x in args.seqlens.split(",")] if args.seqlens else None
+        q, k, v, cu = wl.make_varlen(w, device=dev, seqlens=seqlens)
         out = torch.empty_like(q)
         lse = torch.empty(w.Hq, cu[-1], device=dev, dtype=torch.float32)
         cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
@@ -1182,6 +1232,7 @@ def main():
                          "nothing (a small, self-contained case for ncu captures)")
     ap.add_argument("--L", type=int, default=None, help="with --profile-case: sequence length")
     ap.add_argument("--B", type=int, default=None, help="with --profile-case: batch")
+    ap.add_argument("--seqlens", default=None, help="with --profile-case of a packed workload: its sequence lengths")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

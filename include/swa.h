@@ -279,6 +279,27 @@ int swa_based_linear_decode(const void* q, const void* k, const void* v, float* 
                             int B, int H, int dk, int dv, float scale, int out_dtype, swa_stream_t stream);
 
 /*
+ * One generated token of a Based-style hybrid layer ("Simple linear attention
+ * language models balance the recall-throughput tradeoff", proposed method: a
+ * sliding window and a linear attention side by side) in one launch: the window
+ * branch's swa_cache_append + swa_decode and the linear branch's
+ * swa_based_linear_decode, with the same results as those calls in sequence.
+ *   window branch: q [B, Hq, d], k_new, v_new [B, Hkv, d] bf16 at positions pos
+ *     (DEVICE int32 [B]); the ring cache and sink slots as for swa_cache_append
+ *     (sink_k/sink_v may be NULL when n_sink == 0); out [B, Hq, d] bf16, lse [B, Hq]
+ *     float32 (may be NULL).  Supported: d = 64 and window + n_sink <= 512.
+ *   linear branch: ql, kl [B, H_l, dk], vl [B, H_l, dv] bf16; state, zsum updated in
+ *     place; out_l [B, H_l, dv] bf16.  Supported: dk = 16, dv = 64.
+ * Argument errors return SWA_ERR_INVALID_ARG / SWA_ERR_UNSUPPORTED with nothing
+ * launched; every pointer must be 16-byte aligned (pos and lse 4-byte).
+ */
+int swa_hybrid_decode(const void* q, const void* k_new, const void* v_new, const int32_t* pos,
+                      void* kcache, void* vcache, void* sink_k, void* sink_v, void* out, float* lse,
+                      int B, int Hq, int Hkv, int d, int window, int n_sink, float scale,
+                      const void* ql, const void* kl, const void* vl, float* state, float* zsum,
+                      void* out_l, int H_l, int dk, int dv, float scale_l, swa_stream_t stream);
+
+/*
  * Hadamard output projection, the step after attention ("Rethinking Attention
  * Output Projection: Structured Hadamard Transforms for Efficient Transformers",
  * section 2): per row, z = alpha * (y H) + beta, where H is the fixed Walsh-

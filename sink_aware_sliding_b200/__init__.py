@@ -38,7 +38,7 @@ EXPORTS = (
     "swa_set_wait_timeout_ns", "swa_set_debug_flags", "swa_version", "swa_decode_noalloc",
     "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append", "swa_decode_rope", "swa_bwd",
     "swa_based_linear_state_features", "swa_based_linear_fwd", "swa_based_linear_decode",
-    "swa_decode_ex", "swa_debug_error_word",
+    "swa_decode_ex", "swa_debug_error_word", "swa_hybrid_decode",
 )
 
 _lib = None
@@ -68,6 +68,8 @@ def _load():
     lib.swa_decode_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, SZ, P]
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.swa_hadamard_proj.argtypes = [P, P, P, P, LL, I, I, P]
+    lib.swa_hybrid_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F,
+                                      P, P, P, P, P, P, I, I, I, F, P]
     D = ctypes.c_double
     lib.swa_rope_qk.argtypes = [P, P, P, LL, I, I, I, D, P]
     lib.swa_rope_cache_append.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P]
@@ -84,7 +86,7 @@ def _load():
     lib.swa_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.swa_set_debug_flags.argtypes = [I]
     for name in ("swa_fwd", "swa_fwd_varlen", "swa_cache_fill", "swa_cache_append", "swa_decode",
-                 "swa_decode_ex", "swa_debug_error_word", "swa_decode_noalloc", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
+                 "swa_decode_ex", "swa_debug_error_word", "swa_decode_noalloc", "swa_hybrid_decode", "swa_hadamard_proj", "swa_rope_qk", "swa_rope_cache_append",
                  "swa_decode_rope", "swa_bwd", "swa_based_linear_state_features", "swa_based_linear_fwd",
                  "swa_based_linear_decode",
                  "swa_device_error", "swa_set_debug_flags", "swa_version"):
@@ -334,6 +336,30 @@ def swa_based_linear_decode(q, k, v, state, zsum, out, scale=None, stream=None) 
                                          ctypes.c_float(scale if scale is not None else 1.0 / math.sqrt(dk)), code,
                                          _stream(stream))
     _check(st, "swa_based_linear_decode")
+
+
+def swa_hybrid_decode(q, k_new, v_new, pos, kcache, vcache, sink_k, sink_v, out, lse, window: int, n_sink: int,
+                      ql, kl, vl, state, zsum, out_l, scale=None, scale_l=None, stream=None) -> None:
+    """One hybrid decode step in one launch: the window branch (append k_new/v_new
+    [B, Hkv, d] at pos, decode q [B, Hq, d] into out, lse) and the linear branch
+    (ql, kl [B, H_l, 16], vl [B, H_l, 64]; state/zsum updated; out_l [B, H_l, 64])."""
+    import torch
+    B, Hq, d = q.shape
+    Hkv = kcache.shape[1]
+    H_l, dk = ql.shape[1], ql.shape[2]
+    dv = vl.shape[-1]
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (out, "out"), (ql, "ql"), (kl, "kl"), (vl, "vl"),
+                 (out_l, "out_l")):
+        _need(t.dtype == torch.bfloat16 and t.is_contiguous(), f"{n} bf16 contiguous")
+    _need(state.dtype == torch.float32 and zsum.dtype == torch.float32, "state, zsum float32")
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos int32 [B]")
+    st = _load().swa_hybrid_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(kcache), _ptr(vcache),
+                                   _ptr(sink_k), _ptr(sink_v), _ptr(out), _ptr(lse), B, Hq, Hkv, d, int(window),
+                                   int(n_sink), _scale(scale, d), _ptr(ql), _ptr(kl), _ptr(vl), _ptr(state),
+                                   _ptr(zsum), _ptr(out_l), H_l, dk, dv,
+                                   ctypes.c_float(scale_l if scale_l is not None else 1.0 / math.sqrt(dk)),
+                                   _stream(stream))
+    _check(st, "swa_hybrid_decode")
 
 
 def swa_hadamard_proj(y, alpha, beta, z, stream=None) -> None:

@@ -443,6 +443,53 @@ int swa_bwd(const void* q, const void* k, const void* v, const void* out, const 
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+int swa_hybrid_decode(const void* q, const void* k_new, const void* v_new, const int32_t* pos, void* kcache,
+                      void* vcache, void* sink_k, void* sink_v, void* out, float* lse, int B, int Hq, int Hkv,
+                      int d, int window, int n_sink, float scale, const void* ql, const void* kl, const void* vl,
+                      float* state, float* zsum, void* out_l, int H_l, int dk, int dv, float scale_l,
+                      swa_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || window < 1 || n_sink < 0 || H_l <= 0)
+    return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale) || !(scale_l > 0.f) || !std::isfinite(scale_l))
+    return SWA_ERR_INVALID_ARG;
+  if (!swa::hybrid_window_supported(d, window, n_sink) || dk != 16 || dv != 64) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  const void* ptrs[] = {q, k_new, v_new, kcache, vcache, out, ql, kl, vl, state, zsum, out_l};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return SWA_ERR_INVALID_ARG;
+  if (n_sink > 0 && (!sink_k || !sink_v || !aligned16(sink_k) || !aligned16(sink_v))) return SWA_ERR_INVALID_ARG;
+  if (!pos || (reinterpret_cast<uintptr_t>(pos) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return SWA_ERR_INVALID_ARG;
+  swa::HybridArgs a{};
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.pos = pos;
+  a.kcache = kcache;
+  a.vcache = vcache;
+  a.sink_k = sink_k;
+  a.sink_v = sink_v;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.W = window;
+  a.S = n_sink;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.ql = ql;
+  a.kl = kl;
+  a.vl = vl;
+  a.state = state;
+  a.zsum = zsum;
+  a.out_l = out_l;
+  a.H_l = H_l;
+  a.scale_l = scale_l;
+  cudaError_t e = swa::launch_hybrid_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 int swa_based_linear_state_features(int dk) { return dk > 0 ? swa::based_linear_features(dk) : 0; }
 
 int swa_based_linear_fwd(const void* q, const void* k, const void* v, void* out, float* state, float* zsum,

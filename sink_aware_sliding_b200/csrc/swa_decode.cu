@@ -297,28 +297,32 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 }
 
-// One CTA per (b, kvh) segment and query head h of that KV head, D threads (one output
-// element each): combine the partials of the pieces that covered the segment by their
-// log-sum-exps.  Pieces w_first .. w_last of the concatenated key range overlap the
-// segment (none is empty, see effective_pieces).  The head's maximum over the pieces
-// is reduced first; then the weights exp2(m_w - M) are staged in shared memory a chunk
-// at a time and every thread accumulates its element over them, with the loads of a
-// chunk in flight together.
-template <int D>
-__global__ void __launch_bounds__(D) swa_decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int kChunk = D;
+// One CTA per (b, kvh) segment and query head h of that KV head: combine the partials
+// of the pieces that covered the segment by their log-sum-exps.  Pieces w_first ..
+// w_last of the concatenated key range overlap the segment (none is empty, see
+// effective_pieces).  kMergeSplit x D threads: thread (s, dim) sums output element dim
+// over the pieces p = s mod kMergeSplit, eight loads in flight, so that a segment
+// cut into many pieces (a single long sequence) is not a long chain of dependent
+// loads; the kMergeSplit partial sums are then added in shared memory.  With few
+// pieces per segment (many sequences) kMergeSplit = 1 keeps the CTAs small.
+template <int D, int kMergeSplit>
+__global__ void __launch_bounds__(kMergeSplit * D) swa_decode_merge_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kThreads = kMergeSplit * D;
   const int seg = blockIdx.x;
   const int h = blockIdx.y;
   const int b = seg / a.Hkv, kvh = seg % a.Hkv;
   const int G = a.G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ long long s_red[D / 32][2];
-  __shared__ float s_wmax[D / 32];
-  __shared__ float s_e[kChunk];
-  __shared__ float s_el[kChunk];
+  const int dim = tid % D, split = tid / D;
+  __shared__ long long s_red[kThreads / 32][2];
+  __shared__ float s_wmax[kThreads / 32];
+  __shared__ float s_e[kThreads];
+  __shared__ float s_el[kThreads];
+  __shared__ float s_acc[kMergeSplit][D];
+  __shared__ float s_l[kMergeSplit][D];
   // Offset of this segment in the concatenated key range, and the total.
   long long before = 0, total = 0;
-  for (int i = tid; i < a.B; i += D) {
+  for (int i = tid; i < a.B; i += kThreads) {
     const long long l = seg_len(a.pos[i], a.W, a.S);
     total += l;
     if (i < b) before += l;
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(D) swa_decode_merge_kernel(const __grid_consta
   __syncthreads();
   before = total = 0;
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) {
+  for (int w = 0; w < kThreads / 32; ++w) {
     before += s_red[w][0];
     total += s_red[w][1];
   }
@@ -351,18 +355,18 @@ __global__ void __launch_bounds__(D) swa_decode_merge_kernel(const __grid_consta
 
   // 1. this head's reference max over the pieces
   float m = -INFINITY;
-  for (int p = tid; p < np; p += D) m = fmaxf(m, part0[p * part_floats + G * D + h]);
+  for (int p = tid; p < np; p += kThreads) m = fmaxf(m, part0[p * part_floats + G * D + h]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) s_wmax[warp] = m;
   __syncthreads();
   float M = s_wmax[0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_wmax[w]);
+  for (int w = 1; w < kThreads / 32; ++w) M = fmaxf(M, s_wmax[w]);
 
-  // 2. weighted sums, kChunk pieces at a time
+  // 2. weighted sums, kThreads pieces' weights staged at a time
   float acc = 0.f, lacc = 0.f;
-  for (int c0 = 0; c0 < np; c0 += kChunk) {
+  for (int c0 = 0; c0 < np; c0 += kThreads) {
     {
       const int p = c0 + tid;
       float e = 0.f, el = 0.f;
@@ -375,32 +379,43 @@ __global__ void __launch_bounds__(D) swa_decode_merge_kernel(const __grid_consta
       s_el[tid] = el;
     }
     __syncthreads();
-    const int n = min(kChunk, np - c0);
-    const float* pp = part0 + static_cast<size_t>(c0) * part_floats + h * D + tid;
-    int p = 0;
-    for (; p + 8 <= n; p += 8) {
+    const int n = min(kThreads, np - c0);
+    const float* pp = part0 + static_cast<size_t>(c0) * part_floats + h * D + dim;
+    for (int p0 = split; p0 < n; p0 += 8 * kMergeSplit) {
       float v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = pp[(p + u) * part_floats];
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * kMergeSplit;
+        v[u] = p < n ? pp[p * part_floats] : 0.f;
+      }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        acc += s_e[p + u] * v[u];
-        lacc += s_el[p + u];
+        const int p = p0 + u * kMergeSplit;
+        if (p < n) {
+          acc += s_e[p] * v[u];
+          lacc += s_el[p];
+        }
       }
-    }
-    for (; p < n; ++p) {
-      acc += s_e[p] * pp[p * part_floats];
-      lacc += s_el[p];
     }
     __syncthreads();
   }
-  const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
-  const float o = acc / lacc;
-  if (a.out_f32)
-    static_cast<float*>(a.out)[orow * D + tid] = o;
-  else
-    static_cast<__nv_bfloat16*>(a.out)[orow * D + tid] = __float2bfloat16_rn(o);
-  if (tid == 0 && a.lse != nullptr) a.lse[orow] = (M + log2f(lacc)) * 0.69314718055994531f;
+  s_acc[split][dim] = acc;
+  s_l[split][dim] = lacc;
+  __syncthreads();
+  if (split == 0) {
+#pragma unroll
+    for (int s2 = 1; s2 < kMergeSplit; ++s2) {
+      acc += s_acc[s2][dim];
+      lacc += s_l[s2][dim];
+    }
+    const size_t orow = static_cast<size_t>(b) * a.Hq + kvh * G + h;
+    const float o = acc / lacc;
+    if (a.out_f32)
+      static_cast<float*>(a.out)[orow * D + dim] = o;
+    else
+      static_cast<__nv_bfloat16*>(a.out)[orow * D + dim] = __float2bfloat16_rn(o);
+    if (dim == 0 && a.lse != nullptr) a.lse[orow] = (M + log2f(lacc)) * 0.69314718055994531f;
+  }
 }
 
 template <int D>
@@ -415,7 +430,12 @@ cudaError_t launch_decode_impl(const DecodeArgs& a, int grid, int block, cudaStr
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  swa_decode_merge_kernel<D><<<dim3(a.B * a.Hkv, a.G), D, 0, stream>>>(a);
+  // pieces per segment when the sequences are equally long: the grid's warps over the segments
+  const long long pieces = a.n_warps / (static_cast<long long>(a.B) * a.Hkv) + 1;
+  if (pieces > 16)
+    swa_decode_merge_kernel<D, 4><<<dim3(a.B * a.Hkv, a.G), 4 * D, 0, stream>>>(a);
+  else
+    swa_decode_merge_kernel<D, 1><<<dim3(a.B * a.Hkv, a.G), D, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

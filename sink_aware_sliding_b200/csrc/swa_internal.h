@@ -110,6 +110,33 @@ cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos,
                                void* sk, void* sv, int B, int Hkv, int d, int W, int S,
                                const RopeTable& rt, cudaStream_t stream);
 
+// One hybrid decode step: the window branch (append, decode; d = 64) and the Based
+// linear branch (recurrent step; dk = 16, dv = 64) in one launch.
+struct HybridArgs {
+  const void* q;            // [B, Hq, 64] bf16
+  const void* k_new;        // [B, Hkv, 64] bf16
+  const void* v_new;
+  const int32_t* pos;       // [B]
+  void* kcache;             // [B, Hkv, W, 64] bf16
+  void* vcache;
+  void* sink_k;             // [B, Hkv, S, 64] bf16 (unused when S == 0)
+  void* sink_v;
+  void* out;                // [B, Hq, 64] bf16
+  float* lse;               // [B, Hq] or null
+  int B, Hq, Hkv, G, W, S;
+  float scale_log2;
+  const void* ql;           // [B, H_l, 16] bf16
+  const void* kl;
+  const void* vl;           // [B, H_l, 64] bf16
+  float* state;             // [B, H_l, 273, 64]
+  float* zsum;              // [B, H_l, 273]
+  void* out_l;              // [B, H_l, 64] bf16
+  int H_l;
+  float scale_l;
+};
+bool hybrid_window_supported(int d, int window, int n_sink);
+cudaError_t launch_hybrid_decode(const HybridArgs& a, cudaStream_t stream);
+
 // Hadamard output projection z = alpha * (y H) + beta over rows of n = 2^k elements.
 struct HadamardArgs {
   const void* y;            // [n_rows, n] bf16
