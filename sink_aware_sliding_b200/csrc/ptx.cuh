@@ -41,14 +41,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
+// The suspend-time hint lets a waiting thread sleep until the phase completes (or
+// the hint, in ns, runs out) instead of returning at once: waiting warps then give
+// their issue slots to the working warps of their SM sub-partition (measured on a
+// B200: 2% on the tensor-bound prefill, 5% on the short-window one).
+constexpr uint32_t kWaitSuspendHintNs = 2000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kWaitSuspendHintNs)
       : "memory");
   return ok != 0;
 }

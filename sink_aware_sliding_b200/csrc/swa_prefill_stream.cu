@@ -288,6 +288,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     if (lane == 0 && x < n_range) {
       bool ok = true;
       const uint32_t s_t = tmem + C::tmem_s(x);
+      // one descriptor per operand array, stepped by offsets (slot, sub-tile, k-step)
+      const uint64_t dq0 = kmajor_desc<C::QK_STEPS>(base + C::OFF_Q, kBM, 0);
+      const uint64_t dk0 = kmajor_desc<C::QK_STEPS>(base + C::OFF_KV, C::SUB, 0);
+      const uint64_t dv0 = v_desc<false, C::KSTEP>(base + C::OFF_KV + C::TILE, 0);
       // this warpgroup's 64-key sub-tiles in order: query tiles li = x, x+2, ...,
       // within each the sub-tiles f64 .. l64 of its band
       struct Sub {
@@ -328,12 +332,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         if (u.s64 == u.f64 && !wait_bar(bar(C::B_QFULL + u.li % C::NQ), (u.li / C::NQ) & 1, ctl)) return false;
         if (!wait_bar(bar(C::B_KVFULL + kc % C::NKV), (kc / C::NKV) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t q_tile = base + C::OFF_Q + (u.li % C::NQ) * C::TILE;
-        const uint32_t k_sub = base + C::OFF_KV + (kc % C::NKV) * 2 * C::TILE + (u.s64 & 1) * (C::SUB * 128);
+        const uint64_t dq = desc_add(dq0, (u.li % C::NQ) * C::TILE);
+        const uint64_t dk = desc_add(dk0, (kc % C::NKV) * 2 * C::TILE + (u.s64 & 1) * (C::SUB * 128));
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(s_t + C::SUB * half, kmajor_desc<C::QK_STEPS>(q_tile, kBM, kk),
-                         kmajor_desc<C::QK_STEPS>(k_sub, C::SUB, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_ss<false>(s_t + C::SUB * half, desc_add(dq, kmajor_off<C::QK_STEPS, kBM>(kk)),
+                         desc_add(dk, kmajor_off<C::QK_STEPS, C::SUB>(kk)), C::IDESC_QK, kk > 0 ? 1u : 0u);
         tc_commit(bar(C::B_SFULL + 2 * x + half));
         return true;
       };
@@ -349,13 +353,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
           if (!(ok = wait_bar(bar(C::B_PFULL + 2 * x + (g & 1)), (g >> 1) & 1, ctl))) break;
           tc_fence_after();
           const int kc = kc_of(cur);
-          const uint32_t v_tile = base + C::OFF_KV + (kc % C::NKV) * 2 * C::TILE + C::TILE;
+          const uint64_t dv = desc_add(dv0, (kc % C::NKV) * 2 * C::TILE + (cur.s64 & 1) * (C::SUB * 128));
           const uint32_t o_t = tmem + C::tmem_o(x, cur.k & 1);
 #pragma unroll
           for (int kk = 0; kk < C::PV_STEPS; ++kk)
-            umma_ts<false>(o_t, s_t + C::SUB * (g & 1) + kk * 8,
-                           v_desc<false, C::KSTEP>(v_tile, kk + C::PV_STEPS * (cur.s64 & 1)), C::IDESC_PV,
-                           (cur.s64 == cur.f64 && kk == 0) ? 0u : 1u);
+            umma_ts<false>(o_t, s_t + C::SUB * (g & 1) + kk * 8, desc_add(dv, mnmajor_off<C::KSTEP>(kk)),
+                           C::IDESC_PV, (cur.s64 == cur.f64 && kk == 0) ? 0u : 1u);
           tc_commit(bar(C::B_PVDONE + x));
           if ((cur.s64 & 1) || cur.s64 == cur.l64) {     // this tile's last use of the key tile
             tc_commit(bar(C::B_KVEMPTY + kc % C::NKV));
