@@ -220,6 +220,58 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, const Unit& x, int
   return need;
 }
 
+// Sink mini-tile.  A sink prefix of at most kSinkMini keys whose key tile lies
+// left of the band (the band starts at key 128 or later) is not run as a masked
+// 128-key tile: Q K^T is formed on the first 16 keys only (N = 16), the softmax
+// works on 16 columns, and P V is one K = 16 product.  Every row sees every sink
+// then (rows are past key 127), so the mask is just c < n_sink.  The K and V tiles
+// are still loaded whole; only their first 16 rows are read.
+constexpr int kSinkMini = 16;
+__device__ __forceinline__ bool sink_mini(const Unit& x, int n_sink) {
+  return x.nst == 1 && n_sink <= kSinkMini;
+}
+
+// Online softmax of the sink mini-tile (bf16 path): S columns 0..15 at s_tmem, P
+// (8 packed bf16 pairs) written over columns 0..7.  Same running max, sum and
+// rescale rule as softmax_tile.
+__device__ __forceinline__ bool softmax_sink16(uint32_t s_tmem, int n_sink, float sl2, float& m_run,
+                                               float& l_run, float& alpha) {
+  float s[kSinkMini];
+  {
+    uint32_t sr[kSinkMini];
+    tmem_ld16_wait(s_tmem, sr);
+#pragma unroll
+    for (int c = 0; c < kSinkMini; ++c) s[c] = c < n_sink ? __uint_as_float(sr[c]) : -INFINITY;
+  }
+  float mx[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mx[i] = max3(s[i], s[4 + i], fmaxf(s[8 + i], s[12 + i]));
+  const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  const float m_new = fmaxf(m_run, m_tile);
+  const bool need = (m_new - m_run) * sl2 > 8.0f;
+  const float m_use = need ? m_new : m_run;
+  alpha = need ? ex2_approx((m_run - m_new) * sl2) : 1.0f;
+  const float neg = (m_use == -INFINITY) ? 0.0f : -m_use * sl2;
+  const uint64_t scale2 = f2_pack(sl2, sl2), neg2 = f2_pack(neg, neg);
+  uint64_t acc[2] = {0, 0};
+  uint32_t pr[kSinkMini / 2];
+#pragma unroll
+  for (int i = 0; i < kSinkMini / 2; ++i) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, neg2), x0, x1);
+    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
+    pr[i] = pack_bf16x2(p0, p1);
+  }
+  float sum0, sum1, sum2, sum3;
+  f2_unpack(acc[0], sum0, sum1);
+  f2_unpack(acc[1], sum2, sum3);
+  l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
+  m_run = m_use;
+  tmem_st8(s_tmem, pr);
+  return need;
+}
+
 // Scale this warp's 32 rows of O (d columns at o_tmem) by alpha (per row).
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t o_tmem, float alpha) {

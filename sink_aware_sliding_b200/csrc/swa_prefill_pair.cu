@@ -4,7 +4,9 @@
 // Work unit = (sequence, 128-row query tile, head pair).  Both tiles visit the
 // same key tiles (the band plus the sink prefix, nothing else); when the two
 // heads read the same KV head (grouped-query attention with an even group) the
-// K and V tiles are loaded once for both.
+// K and V tiles are loaded once for both.  A sink prefix of at most 16 keys left
+// of the band is a 16-key mini-tile (sink_mini): its products and softmax cover
+// 16 keys instead of a masked 128-key tile.
 //
 // Roles (384 threads):
 //   warps 0-3   softmax of tile A (thread r = query row r = TMEM lane r)
@@ -74,6 +76,7 @@ struct PairCfg {
   static constexpr int OFF_TABLES = OFF_ABORT + 12;
   static constexpr int SMEM_BYTES = OFF_TABLES + 2 * 4 * (kMaxSeqSmem + 1) + 1024;
   static constexpr uint32_t IDESC_QK = make_idesc(F32 ? 2u : 1u, kBM, kBN, false);
+  static constexpr uint32_t IDESC_QK_SINK = make_idesc(1u, kBM, kSinkMini, false);   // bf16 only
   static constexpr uint32_t IDESC_PV = make_idesc(F32 ? 2u : 1u, kBM, D, true);
   static constexpr bool TMA_STORE = !F32 && D == 64;   // requires QBUF == 2 (see above)
   __device__ static constexpr uint32_t tmem_s(int half) { return half ? 128u : 0u; }
@@ -216,12 +219,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t dq0 = kmajor_desc<SPC>(base + C::OFF_Q, kBM, 0);
       const uint64_t dk0 = kmajor_desc<SPC>(base + C::OFF_RING, kBN, 0);
       const uint64_t dv0 = v_desc<F32, C::KSTEP>(base + C::OFF_RING, 0);
-      auto qk = [&](int half, uint64_t dq, int k_ctr) {
+      auto qk = [&](int half, uint64_t dq, int k_ctr, uint32_t idesc) {
         const uint64_t dk = desc_add(dk0, (k_ctr % C::NSTAGE) * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
           umma_ss<F32>(tmem + C::tmem_s(half), desc_add(dq, kmajor_off<SPC, kBM>(kk)),
-                       desc_add(dk, kmajor_off<SPC, kBN>(kk)), C::IDESC_QK, kk > 0 ? 1u : 0u);
+                       desc_add(dk, kmajor_off<SPC, kBN>(kk)), idesc, kk > 0 ? 1u : 0u);
         tc_commit(bar(C::B_SFULL + half));
       };
       auto pv = [&](int half, int v_ctr, bool first) {
@@ -230,6 +233,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
           umma_ts<F32>(tmem + C::tmem_o(half), tmem + C::tmem_s(half) + kk * 8, desc_add(dv, mnmajor_off<C::KSTEP>(kk)),
                        C::IDESC_PV, (first && kk == 0) ? 0u : 1u);
+      };
+      // P V of the sink mini-tile: one K = 16 step (keys 0..15), starting the accumulator
+      auto pv_sink = [&](int half, int v_ctr) {
+        umma_ts<F32>(tmem + C::tmem_o(half), tmem + C::tmem_s(half), desc_add(dv0, (v_ctr % C::NSTAGE) * C::TILE),
+                     C::IDESC_PV, 0u);
       };
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
         Unit x;
@@ -243,6 +251,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // ring positions in the load order K(0), K(1), V(0), K(2), V(1), ..., V(n-1), in groups
         // of g = per / 2 slots (A, then B when the heads read different KV heads)
         const int g = per / 2, nt = x.n_tiles;
+        const bool mini = !F32 && sink_mini(x, a.n_sink);     // key tile 0 is the sink mini-tile
         auto kA = [&](int j) { return ld + (j == 0 ? 0 : (2 * j - 1) * g); };
         auto kB = [&](int j) { return kA(j) + (shared ? 0 : 1); };
         auto vA = [&](int j) { return ld + (j == nt - 1 ? 2 * nt - 1 : 2 * j + 2) * g; };
@@ -250,12 +259,35 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // prologue: S_A(0), S_B(0)
         if (!(ok = wait_full(kA(0)) && (shared || wait_full(kB(0))))) break;
         tc_fence_after();
-        qk(0, qA, kA(0));
-        qk(1, qB, kB(0));
+        // S(0): Q K^T over the first 16 keys only when key tile 0 is the sink mini-tile
+        qk(0, qA, kA(0), mini ? C::IDESC_QK_SINK : C::IDESC_QK);
+        qk(1, qB, kB(0), mini ? C::IDESC_QK_SINK : C::IDESC_QK);
         tc_commit(bar(C::B_EMPTY + kA(0) % C::NSTAGE));
         if (!shared) tc_commit(bar(C::B_EMPTY + kB(0) % C::NSTAGE));
         if (!kTmaStore && x.n_tiles == 1) tc_commit(bar(C::B_QEMPTY + qb));
-        for (int j = 0; j < x.n_tiles; ++j, ++cnt) {
+        int j0 = 0;
+        if (mini) {
+          // key tile 0 = the sink mini-tile (a mini unit has band tiles after it, so tile 0
+          // is never the last): the same steps as the loop below, with the short P V
+          if (!(ok = wait_bar(bar(C::B_PFULL + 0), cnt & 1, ctl) && wait_full(vA(0)))) break;
+          tc_fence_after();
+          pv_sink(0, vA(0));
+          if (!(ok = wait_full(kA(1)) && (shared || wait_full(kB(1))))) break;
+          tc_fence_after();
+          qk(0, qA, kA(1), C::IDESC_QK);
+          if (!(ok = wait_bar(bar(C::B_PFULL + 1), cnt & 1, ctl) && (shared || wait_full(vB(0))))) break;
+          tc_fence_after();
+          pv_sink(1, vB(0));
+          tc_commit(bar(C::B_EMPTY + vA(0) % C::NSTAGE));
+          if (!shared) tc_commit(bar(C::B_EMPTY + vB(0) % C::NSTAGE));
+          qk(1, qB, kB(1), C::IDESC_QK);
+          tc_commit(bar(C::B_EMPTY + kA(1) % C::NSTAGE));
+          if (!shared) tc_commit(bar(C::B_EMPTY + kB(1) % C::NSTAGE));
+          if (!kTmaStore && x.n_tiles == 2) tc_commit(bar(C::B_QEMPTY + qb));
+          j0 = 1;
+          ++cnt;
+        }
+        for (int j = j0; j < x.n_tiles; ++j, ++cnt) {
           const bool last = j == x.n_tiles - 1;
           // ---- tile A: O_A += P_A(j) V(j), then S_A(j+1)
           if (!(ok = wait_bar(bar(C::B_PFULL + 0), cnt & 1, ctl) && wait_full(vA(j)))) break;
@@ -265,7 +297,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (!last) {
             if (!(ok = wait_full(kA(j + 1)) && (shared || wait_full(kB(j + 1))))) break;
             tc_fence_after();
-            qk(0, qA, kA(j + 1));
+            qk(0, qA, kA(j + 1), C::IDESC_QK);
           }
           // ---- tile B: O_B += P_B(j) V(j), then S_B(j+1)
           if (!(ok = wait_bar(bar(C::B_PFULL + 1), cnt & 1, ctl) && (shared || wait_full(vB(j))))) break;
@@ -276,7 +308,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (last) {
             tc_commit(bar(C::B_OFINAL + 1));
           } else {
-            qk(1, qB, kB(j + 1));
+            qk(1, qB, kB(j + 1), C::IDESC_QK);
             tc_commit(bar(C::B_EMPTY + kA(j + 1) % C::NSTAGE));
             if (!shared) tc_commit(bar(C::B_EMPTY + kB(j + 1) % C::NSTAGE));
             if (!kTmaStore && j + 1 == x.n_tiles - 1) tc_commit(bar(C::B_QEMPTY + qb));
@@ -309,7 +341,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       unit_of(u, x, hA);
       const int t = x.m0 + r;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < x.n_tiles; ++j, ++cnt) {
+      int j0 = 0;
+      if (!F32 && sink_mini(x, a.n_sink)) {
+        // key tile 0 = the sink mini-tile: the first tile of the unit, so O needs no rescale
+        ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SFULL + half), cnt & 1, ctl));
+        if (!ok) break;
+        tc_fence_after();
+        float alpha;
+        softmax_sink16(s_tmem, a.n_sink, a.scale_log2, m_run, l_run, alpha);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + half));
+        j0 = 1;
+        ++cnt;
+      }
+      for (int j = j0; j < x.n_tiles; ++j, ++cnt) {
         ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SFULL + half), cnt & 1, ctl));
         if (!ok) break;
         tc_fence_after();

@@ -87,6 +87,10 @@ def test_tiny_workload_fp32():
     (1, 500, 4, 2, 128, 40, 4),        # sink tile is the first band tile
     (1, 500, 4, 2, 64, 40, 70),        # sink prefix across the first band tile, d = 64
     (2, 640, 4, 2, 64, 200, 4),        # d = 64 GQA: TMA-store epilogue over several units
+    (1, 900, 4, 2, 128, 256, 16),      # 16 sinks: the widest sink mini-tile
+    (1, 900, 4, 2, 64, 256, 17),       # 17 sinks: a whole masked sink tile again
+    (1, 700, 4, 4, 128, 200, 1),       # a single sink
+    (1, 1200, 2, 1, 64, 300, 16),      # mini-tile at d = 64 with the TMA-store epilogue
 ])
 def test_prefill_matches_oracle(B, L, Hq, Hkv, d, window, n_sink):
     q, k, v = rand_qkv(B, L, Hq, Hkv, d, seed=B * 1000 + L)
