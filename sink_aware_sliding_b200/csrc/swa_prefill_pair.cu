@@ -289,18 +289,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         for (int j = j0; j < x.n_tiles; ++j, ++cnt) {
           const bool last = j == x.n_tiles - 1;
+          // The data tiles first: they were requested a tile or more ahead and are in by
+          // now, and checking them while P_A is still being written keeps those checks
+          // (about 200 cycles each, measured) off the P -> MMA path.
+          if (!(ok = wait_full(vA(j)) && (shared || wait_full(vB(j))))) break;
+          if (!last && !(ok = wait_full(kA(j + 1)) && (shared || wait_full(kB(j + 1))))) break;
           // ---- tile A: O_A += P_A(j) V(j), then S_A(j+1)
-          if (!(ok = wait_bar(bar(C::B_PFULL + 0), cnt & 1, ctl) && wait_full(vA(j)))) break;
+          if (!(ok = wait_bar(bar(C::B_PFULL + 0), cnt & 1, ctl))) break;
           tc_fence_after();
           pv(0, vA(j), j == 0);
           if (last) tc_commit(bar(C::B_OFINAL + 0));
-          if (!last) {
-            if (!(ok = wait_full(kA(j + 1)) && (shared || wait_full(kB(j + 1))))) break;
-            tc_fence_after();
-            qk(0, qA, kA(j + 1), C::IDESC_QK);
-          }
+          if (!last) qk(0, qA, kA(j + 1), C::IDESC_QK);
           // ---- tile B: O_B += P_B(j) V(j), then S_B(j+1)
-          if (!(ok = wait_bar(bar(C::B_PFULL + 1), cnt & 1, ctl) && (shared || wait_full(vB(j))))) break;
+          if (!(ok = wait_bar(bar(C::B_PFULL + 1), cnt & 1, ctl))) break;
           tc_fence_after();
           pv(1, vB(j), j == 0);
           tc_commit(bar(C::B_EMPTY + vA(j) % C::NSTAGE));
