@@ -18,19 +18,21 @@
 // A third, small kernel computes D_t = rowsum(dO_t O_t) for every row first,
 // into the storage of dq (which the dQ kernel only writes after the dK/dV kernel
 // has read D; the dQ kernel forms its own D per row).
-// Each CTA is two warpgroups over the same 128 TMEM lanes: the first does the
-// element-wise step on score columns 0-63, the second on columns 64-127 (the step
-// is independent per column), so each thread handles half a row.  Visibility is
-// tested only on edge tiles, through four 32-bit words per row built from the row's
-// visible column ranges.  Thread 0 issues TMA and MMA; every hand-off is an
-// mbarrier with a bounded wait.  Thread 0
-// shares warp 0 with element-wise threads, so the warp is reconverged
-// (__syncwarp) after every issuer-only block and every wait's outcome is made
-// warp-uniform before the warp-collective tcgen05 instructions that follow.  The
-// tiles that change per iteration (Q and dO, or K and V) are double-buffered and
-// the next iteration's are requested when the current one starts; the products
-// and the element-wise step of one iteration still run one after another (TMEM
-// holds one iteration's S^T and dP^T next to the accumulators).
+// Each CTA has two element-wise warpgroups over the same 128 TMEM lanes: the first
+// does the element-wise step on score columns 0-63, the second on columns 64-127
+// (the step is independent per column), so each thread handles half a row.
+// Visibility is tested only on edge tiles, through four 32-bit words per row built
+// from the row's visible column ranges.  Every hand-off is an mbarrier with a
+// bounded wait.  In the dK/dV kernel a ninth warp issues TMA and MMA and stages the
+// per-row data, so the products of one iteration and the scores of the next go out
+// back to back (see the kernel).  In the dQ kernel thread 0 issues TMA and MMA and
+// shares warp 0 with element-wise threads, so the warp is reconverged (__syncwarp)
+// after every issuer-only block and every wait's outcome is made warp-uniform before
+// the warp-collective tcgen05 instructions that follow; its tiles that change per
+// iteration (K and V) are double-buffered and the next iteration's are requested when
+// the current one starts.  In both, the products and the element-wise step of one
+// iteration still run one after another (TMEM holds one iteration's scores next to
+// the accumulators).
 //
 // TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
 // written over their first halves), dV 256.., dK 256+d..; (dQ kernel): S 0-127,
@@ -50,7 +52,7 @@ namespace {
 using namespace prefill;
 
 constexpr int kBwdThreads = 256;
-constexpr int kRowThreads = 128;   // the first warpgroup also stages the per-row data
+constexpr int kEwThreads = 256;    // dK/dV kernel: the element-wise threads (warps 0-7)
 
 template <int D>
 struct BwdCfg {
@@ -58,15 +60,12 @@ struct BwdCfg {
   static constexpr int NCHUNK = D / 64;                // 128-byte column chunks
   static constexpr int QK_STEPS = D / 16;
   static constexpr int PV_STEPS = kBN / 16;
-  // shared layout: tiles 0..5 (two fixed, two double-buffered), then D_s, L_s
-  // (128 floats each), the next iterations' D and lse as copied (two buffers of
-  // 128 + 128 floats), then barriers
+  // shared layout: tiles 0..5 (two fixed, two double-buffered), then the dK/dV
+  // kernel's row data (two slots of 128 D + 128 lse floats), then barriers
   static constexpr int OFF_T = 0;
-  static constexpr int OFF_DS = 6 * TILE;
-  static constexpr int OFF_LS = OFF_DS + 512;
-  static constexpr int OFF_STG = OFF_LS + 512;
+  static constexpr int OFF_STG = 6 * TILE;
   static constexpr int OFF_BAR = OFF_STG + 2048;
-  static constexpr int NBAR = 8;
+  static constexpr int NBAR = 9;
   static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
   // Each CTA allocates all 512 TMEM columns, so no second CTA may share the SM
   // (its allocation would have to wait): ask for more than half of the SM's
@@ -81,10 +80,11 @@ struct BwdCfg {
 constexpr int kBarA = 0;      // K,V (dK/dV kernel) or Q,dO (dQ kernel): loaded once
 constexpr int kBarB = 1;      // the per-iteration tile pair, buffers 0 and 1 (kBarB, kBarB + 1)
 constexpr int kBarS = 3;      // both score products done
-constexpr int kBarP = 4;      // all 128 rows wrote their P / dS (count 128)
+constexpr int kBarP = 4;      // every element-wise thread wrote its P / dS
 constexpr int kBarO = 5;      // accumulation products done
-constexpr int kBarRow = 6;    // per-iteration row data (D, lse) written (count 128)
+constexpr int kBarRow = 6;    // dK/dV kernel: row data (D, lse) of even iterations staged
 constexpr int kBarDrain = 7;
+constexpr int kBarRow2 = 8;   // dK/dV kernel: row data of odd iterations staged
 
 __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const PrefillArgs& a) {
   for (int i = 0; i < 256; ++i)
@@ -150,8 +150,23 @@ __global__ void __launch_bounds__(256) swa_bwd_dot_kernel(const __grid_constant_
 }
 
 // ------------------------------------------------------------------ dK, dV
+// Roles (288 threads): warps 0-7 the element-wise step (warpgroup 0 on score
+// columns 0-63, warpgroup 1 on 64-127; thread = TMEM lane = key row); warp 8 the
+// producer, whose lane 0 issues the TMA loads and the MMAs and whose 32 lanes copy
+// the per-row data (D and lse) into a two-slot staging buffer.  For iteration it
+// the producer waits until every element-wise thread has written P^T(it) and
+// dS^T(it), issues dV += P^T dO and dK += dS^T Q and right behind them S^T and dP^T
+// of iteration it + 1 (the tensor pipe runs in issue order, so those overwrite P^T
+// and dS^T only after the accumulation has read them), copies the row data of
+// it + 2 into the slot iteration it has finished reading, publishes the row data
+// of it + 1, and, once the accumulation of it is done reading Q and dO, requests the
+// tiles of it + 2 into that buffer.  The element-wise warps wait only for their
+// iteration's row data and scores.
+constexpr int kDkdvThreads = 288;
+constexpr int kDkdvProducerWarp = 8;
+
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDkdvThreads, 1)
     swa_bwd_dkdv_kernel(const __grid_constant__ BwdArgs ba, const __grid_constant__ CUtensorMap tq,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                         const __grid_constant__ CUtensorMap tdo) {
@@ -163,10 +178,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8 * i; };
   const uint32_t sK = base + C::OFF_T, sV = sK + C::TILE, sQ = sV + C::TILE, sdO = sQ + C::TILE;
-  float* D_s = reinterpret_cast<float*>(gbase + C::OFF_DS);
-  float* L_s = reinterpret_cast<float*>(gbase + C::OFF_LS);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
 
   const int tiles = (a.L + kBM - 1) / kBM;
   const int jt = blockIdx.x % tiles;
@@ -178,11 +192,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < C::NBAR; ++i)
-      mbar_init(bar(i), i == kBarP ? kBwdThreads : (i == kBarRow ? kRowThreads : 1));
+      mbar_init(bar(i), i == kBarP ? kEwThreads : (i == kBarRow || i == kBarRow2 ? 32 : 1));
     fence_mbar_init();
   }
-  __syncwarp();
-  if (tid < 32) {
+  if (warp == 0) {
     tmem_alloc(smem_u32(tmem_ptr), 512);
     tmem_relinquish();
   }
@@ -190,10 +203,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const int r = tid & 127;                            // TMEM lane (key row) of this thread
-  const int half = tid >> 7;                          // score columns 64 half .. 64 half + 63
-  const bool stager = tid < kRowThreads;
-  const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
   const size_t row_base = static_cast<size_t>(b) * a.L;
 
   // iterations: (query head g, query tile) flattened, query tiles fastest
@@ -201,174 +210,221 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int n_it = a.G * nq;
   auto it_head = [&](int i) { return kvh * a.G + i / nq; };
   auto it_row0 = [&](int i) { return (jt + i % nq) * kBM; };
-  auto issue = [&](int i) {                           // thread 0: Q, dO of iteration i
-    const int buf = i & 1;
-    mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
-    load_tile<D>(sQ + 2 * buf * C::TILE, &tq, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
-    load_tile<D>(sdO + 2 * buf * C::TILE, &tdo, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
-  };
-  const float* d_rows = ba.dq;                        // D, written by the D kernel
-  auto fetch_row = [&](int i, float& dt, float& l2) { // D and lse (log2 units) of query it_row0(i) + r
-    const int t = it_row0(i) + r;
-    const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + t;
-    dt = t < a.L ? d_rows[idx] : 0.f;
-    l2 = t < a.L ? ba.lse[idx] * 1.4426950408889634f : 0.f;
-  };
-  // The same values for a later iteration, copied asynchronously into staging
-  // buffer i & 1 (zero past the sequence's end): a barrier wait that follows loads
-  // into registers would wait for them to land.
-  const uint32_t stg = smem_u32(gbase + C::OFF_STG);
-  auto stage_row = [&](int i) {
-    const int t = it_row0(i) + r;
-    const bool in = t < a.L;
-    const size_t idx = (static_cast<size_t>(b) * a.Hq + it_head(i)) * a.L + (in ? t : 0);
-    const uint32_t dst = stg + (i & 1) * 1024 + r * 4;
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(d_rows + idx), "r"(in ? 4u : 0u)
-                 : "memory");
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 512), "l"(ba.lse + idx), "r"(in ? 4u : 0u)
-                 : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-
+  // staging slot i & 1 of the row data: D at floats 0..127, lse (log2 units) at 128..255
+  auto row_bar = [&](int i) { return bar((i & 1) ? kBarRow2 : kBarRow); };
   bool ok = true;
-  int issued = 0;                                     // iterations whose tiles were requested
-  if (tid == 0) {
-    mbar_expect_tx(bar(kBarA), 2 * C::TILE);
-    load_tile<D>(sK, &tk, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
-    load_tile<D>(sV, &tv, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
-    issue(0);
-    issued = 1;
-  }
-  if (stager) {
-    float next_d = 0.f, next_l = 0.f;
-    fetch_row(0, next_d, next_l);
-    D_s[r] = next_d;
-    L_s[r] = next_l;
-    mbar_arrive(bar(kBarRow));
-  }
-  const int s_key = j0 + r;                           // this thread's key (TMEM lane)
-  // query rows that see this key: s_key .. s_key + window - 1 (all later rows for a
-  // sink), before the sequence's end
-  const int t_hi = min(a.L - 1, s_key < a.n_sink ? a.L - 1 : s_key + a.window - 1);
-  int it = 0;
-  for (; it < n_it; ++it) {
-    const int i0 = it_row0(it), buf = it & 1;
-    const uint32_t cQ = sQ + 2 * buf * C::TILE, cdO = sdO + 2 * buf * C::TILE;
-    // the next iteration's tiles (its buffer's last readers finished with the
-    // previous iteration) and row data (kept in registers until this one is done)
-    if (tid == 0 && it + 1 < n_it) {
-      issue(it + 1);
-      issued = it + 2;
-    }
-    if (stager && it + 1 < n_it) stage_row(it + 1);
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarRow), it & 1, a)))) break;
-    if (tid == 0) {
-      ok = (it > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB + buf), (it >> 1) & 1, a);
-      if (ok) {
-        tc_fence_after();
+
+  if (warp == kDkdvProducerWarp) {
+    const float* d_rows = ba.dq;                      // D, written by the D kernel
+    const uint32_t stg = smem_u32(gbase + C::OFF_STG);
+    // lane l copies rows l, l + 32, l + 64, l + 96 of iteration i (zero past the end)
+    auto stage_rows = [&](int i) {
+      const int h = it_head(i), t0 = it_row0(i);
+      const uint32_t dst = stg + (i & 1) * 1024;
 #pragma unroll
-        for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem, kmajor_desc<4>(sK, kBN, kk), kmajor_desc<4>(cQ, kBM, kk), C::IDESC_SS,
-                         kk > 0 ? 1u : 0u);
+      for (int m = 0; m < 4; ++m) {
+        const int rr = lane + 32 * m, t = t0 + rr;
+        const bool in = t < a.L;
+        const size_t idx = (static_cast<size_t>(b) * a.Hq + h) * a.L + (in ? t : 0);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + rr * 4), "l"(d_rows + idx),
+                     "r"(in ? 4u : 0u) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 512 + rr * 4), "l"(ba.lse + idx),
+                     "r"(in ? 4u : 0u) : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // once this lane's copies of iteration i have landed: lse to log2 units, publish
+    auto publish_rows = [&](int i) {
+      float* l2 = reinterpret_cast<float*>(gbase + C::OFF_STG + (i & 1) * 1024) + 128;
 #pragma unroll
-        for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem + 128, kmajor_desc<4>(sV, kBN, kk), kmajor_desc<4>(cdO, kBM, kk), C::IDESC_SS,
-                         kk > 0 ? 1u : 0u);
-        tc_commit(bar(kBarS));
+      for (int m = 0; m < 4; ++m) l2[lane + 32 * m] *= 1.4426950408889634f;
+      mbar_arrive(row_bar(i));
+    };
+    // one descriptor per operand array, stepped by offsets (buffer, k-step)
+    const uint64_t dK0 = kmajor_desc<4>(sK, kBN, 0), dV0 = kmajor_desc<4>(sV, kBN, 0);
+    const uint64_t dQ0 = kmajor_desc<4>(sQ, kBM, 0), ddO0 = kmajor_desc<4>(sdO, kBM, 0);
+    const uint64_t vQ0 = v_desc<false, 16>(sQ, 0), vdO0 = v_desc<false, 16>(sdO, 0);
+    auto load_qdo = [&](int i) {                      // lane 0: Q, dO of iteration i into buffer i & 1
+      const int buf = i & 1;
+      mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
+      load_tile<D>(sQ + 2 * buf * C::TILE, &tq, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
+      load_tile<D>(sdO + 2 * buf * C::TILE, &tdo, bar(kBarB + buf), it_head(i), static_cast<int>(row_base) + it_row0(i));
+    };
+    auto scores = [&](int i) {                        // lane 0: S^T = K Q^T, dP^T = V dO^T of iteration i
+      const uint32_t off = 2 * (i & 1) * C::TILE;
+#pragma unroll
+      for (int kk = 0; kk < C::QK_STEPS; ++kk)
+        umma_ss<false>(tmem, desc_add(dK0, kmajor_off<4, kBN>(kk)), desc_add(dQ0, off + kmajor_off<4, kBM>(kk)),
+                       C::IDESC_SS, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < C::QK_STEPS; ++kk)
+        umma_ss<false>(tmem + 128, desc_add(dV0, kmajor_off<4, kBN>(kk)), desc_add(ddO0, off + kmajor_off<4, kBM>(kk)),
+                       C::IDESC_SS, kk > 0 ? 1u : 0u);
+      tc_commit(bar(kBarS));
+    };
+    auto accumulate = [&](int i) {                    // lane 0: dV += P^T dO, dK += dS^T Q of iteration i
+      const uint32_t off = 2 * (i & 1) * C::TILE;
+#pragma unroll
+      for (int kk = 0; kk < C::PV_STEPS; ++kk)
+        umma_ts<false>(tmem + 256, tmem + kk * 8, desc_add(vdO0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+                       (i == 0 && kk == 0) ? 0u : 1u);
+#pragma unroll
+      for (int kk = 0; kk < C::PV_STEPS; ++kk)
+        umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, desc_add(vQ0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+                       (i == 0 && kk == 0) ? 0u : 1u);
+      tc_commit(bar(kBarO));
+    };
+
+    int issued = 0, waited = 0;                       // Q/dO loads requested / their arrivals seen
+    if (lane == 0) {
+      mbar_expect_tx(bar(kBarA), 2 * C::TILE);
+      load_tile<D>(sK, &tk, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
+      load_tile<D>(sV, &tv, bar(kBarA), kvh, static_cast<int>(row_base) + j0);
+      load_qdo(0);
+      issued = 1;
+      if (n_it > 1) {
+        load_qdo(1);
+        issued = 2;
       }
     }
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), it & 1, a)))) break;
-    tc_fence_after();
-    // P^T and dS^T of this key row over this warpgroup's 64 query columns
-    {
-      // every (key, query) pair of the tile visible: no test per column
-      const bool full = j0 + kBN - 1 <= i0 && i0 + kBM - 1 < a.L &&
-                        (j0 >= i0 + kBM - a.window || j0 + kBN - 1 < a.n_sink);
-      uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
-      if (!full) visible_words(s_key - i0, t_hi - i0, -1, vw);
-      uint32_t sr[64], dr[64];
-      tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
-      tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
-      uint32_t pw[32], dw[32];
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float p[2], ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 64 * half + c + e;
-          const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]);
-          p[e] = word_bit(vw, col) ? pe : 0.f;
-          ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
-        }
-        pw[c / 2] = pack_bf16x2(p[0], p[1]);
-        dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
-      }
-      tmem_st32(tmem + lane_off + 32 * half, pw);
-      tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(bar(kBarP));
-    if (tid == 0) {
-      if ((ok = bwd_wait(bar(kBarP), it & 1, a))) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(cdO, kk), C::IDESC_ACC,
-                         (it == 0 && kk == 0) ? 0u : 1u);
-#pragma unroll
-        for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, v_desc<false, 16>(cQ, kk), C::IDESC_ACC,
-                         (it == 0 && kk == 0) ? 0u : 1u);
-        tc_commit(bar(kBarO));
-      }
-    }
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), it & 1, a)))) break;
-    // every thread is past this iteration's element-wise step: publish the next row data
-    if (stager && it + 1 < n_it) {
+    stage_rows(0);
+    if (n_it > 1) {
+      stage_rows(1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
       asm volatile("cp.async.wait_group 0;" ::: "memory");
-      const float* st = reinterpret_cast<const float*>(gbase + C::OFF_STG + ((it + 1) & 1) * 1024);
-      D_s[r] = st[r];
-      L_s[r] = st[128 + r] * 1.4426950408889634f;
-      mbar_arrive(bar(kBarRow));
     }
-  }
-  if (!ok && tid == 0) {
-    // let everything this thread started finish before the CTA releases its memory
-    tc_commit(bar(kBarDrain));
-    bwd_wait(bar(kBarDrain), 0, a);
-    bwd_wait(bar(kBarA), 0, a);
-    for (int i = it; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
-  }
-  __syncwarp();
-  tc_fence_after();
-  if (__all_sync(0xffffffffu, ok)) {        // warp-uniform: the TMEM loads are warp-collective
-    const bool row_ok = s_key < a.L;
-    float* dv = ba.dv + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
-    float* dk = ba.dk + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
-#pragma unroll 1
-    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
-      uint32_t rv[32], rk[32];
-      tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, rv);
-      tmem_ld32_wait(tmem + lane_off + 256 + D + 32 * c, rk);
-      if (!row_ok) continue;
+    publish_rows(0);
+    if (lane == 0) {
+      ok = bwd_wait(bar(kBarA), 0, a) && bwd_wait(bar(kBarB), 0, a);
+      if (ok) {
+        waited = 1;
+        tc_fence_after();
+        scores(0);
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    for (int it = 0; ok && it < n_it; ++it) {
+      // every element-wise thread has written P^T(it) and dS^T(it)
+      if (!(ok = bwd_wait(bar(kBarP), it & 1, a))) break;
+      if (lane == 0) {
+        tc_fence_after();
+        accumulate(it);
+        if (it + 1 < n_it) {
+          ok = bwd_wait(bar(kBarB + ((it + 1) & 1)), ((it + 1) >> 1) & 1, a);
+          if (ok) {
+            waited = it + 2;
+            tc_fence_after();
+            scores(it + 1);
+          }
+        }
+      }
+      if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+      // slot it & 1 is free (every thread is past iteration it): copy it + 2 into it
+      if (it + 2 < n_it) {
+        stage_rows(it + 2);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      if (it + 1 < n_it) publish_rows(it + 1);
+      if (lane == 0 && it + 2 < n_it) {
+        // the accumulation of it read Q and dO from buffer it & 1
+        if ((ok = bwd_wait(bar(kBarO), it & 1, a))) {
+          load_qdo(it + 2);
+          issued = it + 3;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (lane == 0) {
+      // Every product is issued: the drain barrier completes (its only phase) when all
+      // have finished, which is when the element-wise warps read the accumulators.
+      tc_commit(bar(kBarDrain));
+      if (!ok) {
+        // let everything this thread started finish before the CTA releases its memory
+        bwd_wait(bar(kBarDrain), 0, a);
+        bwd_wait(bar(kBarA), 0, a);
+        for (int i = waited; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int r = tid & 127;                          // TMEM lane (key row) of this thread
+    const int half = tid >> 7;                        // score columns 64 half .. 64 half + 63
+    const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
+    const int s_key = j0 + r;                         // this thread's key (TMEM lane)
+    // query rows that see this key: s_key .. s_key + window - 1 (all later rows for a
+    // sink), before the sequence's end
+    const int t_hi = min(a.L - 1, s_key < a.n_sink ? a.L - 1 : s_key + a.window - 1);
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = it_row0(it);
+      if (!(ok = __all_sync(0xffffffffu, bwd_wait(row_bar(it), (it >> 1) & 1, a) &&
+                                             bwd_wait(bar(kBarS), it & 1, a))))
+        break;
+      tc_fence_after();
+      const float* D_s = reinterpret_cast<const float*>(gbase + C::OFF_STG + (it & 1) * 1024);
+      const float* L_s = D_s + 128;
+      // P^T and dS^T of this key row over this warpgroup's 64 query columns
+      {
+        // every (key, query) pair of the tile visible: no test per column
+        const bool full = j0 + kBN - 1 <= i0 && i0 + kBM - 1 < a.L &&
+                          (j0 >= i0 + kBM - a.window || j0 + kBN - 1 < a.n_sink);
+        uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
+        if (!full) visible_words(s_key - i0, t_hi - i0, -1, vw);
+        uint32_t sr[64], dr[64];
+        tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
+        tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
+        uint32_t pw[32], dw[32];
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        *reinterpret_cast<float4*>(dv + 32 * c + i) = make_float4(
-            __uint_as_float(rv[i]), __uint_as_float(rv[i + 1]), __uint_as_float(rv[i + 2]), __uint_as_float(rv[i + 3]));
-        *reinterpret_cast<float4*>(dk + 32 * c + i) =
-            make_float4(__uint_as_float(rk[i]) * a.scale, __uint_as_float(rk[i + 1]) * a.scale,
-                        __uint_as_float(rk[i + 2]) * a.scale, __uint_as_float(rk[i + 3]) * a.scale);
+        for (int c = 0; c < 64; c += 2) {
+          float p[2], ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 64 * half + c + e;
+            const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]);
+            p[e] = word_bit(vw, col) ? pe : 0.f;
+            ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
+          }
+          pw[c / 2] = pack_bf16x2(p[0], p[1]);
+          dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st32(tmem + lane_off + 32 * half, pw);
+        tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+    }
+    // all products done (a single-phase barrier: no parity can be confused with another)
+    ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarDrain), 0, a));
+    tc_fence_after();
+    if (ok) {                                 // warp-uniform: the TMEM loads are warp-collective
+      const bool row_ok = s_key < a.L;
+      float* dv = ba.dv + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
+      float* dk = ba.dk + ((row_base + (row_ok ? s_key : 0)) * a.Hkv + kvh) * D;
+#pragma unroll 1
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
+        uint32_t rv[32], rk[32];
+        tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, rv);
+        tmem_ld32_wait(tmem + lane_off + 256 + D + 32 * c, rk);
+        if (!row_ok) continue;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          *reinterpret_cast<float4*>(dv + 32 * c + i) = make_float4(
+              __uint_as_float(rv[i]), __uint_as_float(rv[i + 1]), __uint_as_float(rv[i + 2]), __uint_as_float(rv[i + 3]));
+          *reinterpret_cast<float4*>(dk + 32 * c + i) =
+              make_float4(__uint_as_float(rk[i]) * a.scale, __uint_as_float(rk[i + 1]) * a.scale,
+                          __uint_as_float(rk[i + 2]) * a.scale, __uint_as_float(rk[i + 3]) * a.scale);
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid < 32) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ dQ
@@ -552,7 +608,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
   static int checked = 0;
   if (!checked) {
     int n1 = 0, n2 = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, swa_bwd_dkdv_kernel<D>, kBwdThreads, C::SMEM_BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, swa_bwd_dkdv_kernel<D>, kDkdvThreads, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kBwdThreads, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -563,7 +619,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
   swa_bwd_dot_kernel<D><<<static_cast<unsigned>(std::min<long long>((rows + 255) / 256, 148LL * 32)), 256, 0, stream>>>(ba);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
+  swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kDkdvThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
