@@ -22,20 +22,18 @@
 // does the element-wise step on score columns 0-63, the second on columns 64-127
 // (the step is independent per column), so each thread handles half a row.
 // Visibility is tested only on edge tiles, through four 32-bit words per row built
-// from the row's visible column ranges.  Every hand-off is an mbarrier with a
-// bounded wait.  In the dK/dV kernel a ninth warp issues TMA and MMA and stages the
-// per-row data, so the products of one iteration and the scores of the next go out
-// back to back (see the kernel).  In the dQ kernel thread 0 issues TMA and MMA and
-// shares warp 0 with element-wise threads, so the warp is reconverged (__syncwarp)
-// after every issuer-only block and every wait's outcome is made warp-uniform before
-// the warp-collective tcgen05 instructions that follow; its tiles that change per
-// iteration (K and V) are double-buffered and the next iteration's are requested when
-// the current one starts.  In both, the products and the element-wise step of one
-// iteration still run one after another (TMEM holds one iteration's scores next to
-// the accumulators).
+// from the row's visible column ranges (a separate code path for fully visible
+// tiles).  Every hand-off is an mbarrier with a bounded wait.  In both kernels a
+// ninth warp issues TMA and MMA, so the accumulation products of one iteration and
+// the score products of the next go out back to back and the element-wise warps
+// wait only for their scores; the tiles that change per iteration (Q and dO, or K
+// and V) are double-buffered and requested two iterations ahead.  The products and
+// the element-wise step of one iteration still run one after another (TMEM holds
+// one iteration's scores next to the accumulators).
 //
 // TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
-// written over their first halves), dV 256.., dK 256+d..; (dQ kernel): S 0-127,
+// written over columns 0-31 and 64-95 of each, every warpgroup within the columns
+// it read), dV 256.., dK 256+d..; (dQ kernel): S 0-127 (dS packed the same way),
 // dP 128-255, dQ 256...
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -51,7 +49,6 @@ namespace {
 
 using namespace prefill;
 
-constexpr int kBwdThreads = 256;
 constexpr int kEwThreads = 256;    // dK/dV kernel: the element-wise threads (warps 0-7)
 
 template <int D>
@@ -125,6 +122,58 @@ __device__ __forceinline__ void visible_words(int lo, int hi, int sk_hi, uint32_
 }
 __device__ __forceinline__ bool word_bit(const uint32_t* w, int c) {
   return static_cast<int>(w[c >> 5] << (31 - (c & 31))) < 0;
+}
+
+// TMEM column of K-step kk (16 score columns, 8 packed bf16 columns) of the packed
+// P / dS operand.  Each warpgroup writes its 64 columns packed into the first 32 of
+// the 64 it read (never into the other warpgroup's, which may still be unread):
+// steps 0-3 at columns 0-31, steps 4-7 at 64-95.
+__host__ __device__ constexpr uint32_t packed_col(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
+
+// Element-wise step of the dK/dV kernel for one key row over 64 query columns
+// col0 .. col0 + 63: P^T = exp2(S^T scale log2 e - lse log2 e) (zero where the pair
+// is not visible, tested only when MASK), dS^T = P^T (dP^T - D); D and the log2 lse
+// of the columns come from shared memory four at a time.  Packed bf16 pairs out.
+template <bool MASK>
+__device__ __forceinline__ void dkdv_elementwise(const uint32_t* sr, const uint32_t* dr, const float* D_s,
+                                                 const float* L_s, float sl2, const uint32_t* vw, int col0,
+                                                 uint32_t* pw, uint32_t* dw) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 4) {
+    const float4 l4 = *reinterpret_cast<const float4*>(L_s + col0 + c);
+    const float4 d4 = *reinterpret_cast<const float4*>(D_s + col0 + c);
+    const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+    float p[4], ds[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float pe = ex2_approx(fmaf(__uint_as_float(sr[c + e]), sl2, -lv[e]));
+      if (MASK) pe = word_bit(vw, col0 + c + e) ? pe : 0.f;
+      p[e] = pe;
+      ds[e] = pe * (__uint_as_float(dr[c + e]) - dv[e]);
+    }
+    pw[c / 2] = pack_bf16x2(p[0], p[1]);
+    pw[c / 2 + 1] = pack_bf16x2(p[2], p[3]);
+    dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+    dw[c / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+  }
+}
+
+// Element-wise step of the dQ kernel for one query row (its D and log2 lse in
+// registers) over 64 key columns col0 .. col0 + 63: dS = P (dP - D).
+template <bool MASK>
+__device__ __forceinline__ void dq_elementwise(const uint32_t* sr, const uint32_t* dr, float dt, float l2,
+                                               float sl2, const uint32_t* vw, int col0, uint32_t* dw) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float ds[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float pe = ex2_approx(fmaf(__uint_as_float(sr[c + e]), sl2, -l2));
+      if (MASK) pe = word_bit(vw, col0 + c + e) ? pe : 0.f;
+      ds[e] = pe * (__uint_as_float(dr[c + e]) - dt);
+    }
+    dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+  }
 }
 
 template <int D>
@@ -266,12 +315,12 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       const uint32_t off = 2 * (i & 1) * C::TILE;
 #pragma unroll
       for (int kk = 0; kk < C::PV_STEPS; ++kk)
-        umma_ts<false>(tmem + 256, tmem + kk * 8, desc_add(vdO0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+        umma_ts<false>(tmem + 256, tmem + packed_col(kk), desc_add(vdO0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
                        (i == 0 && kk == 0) ? 0u : 1u);
 #pragma unroll
       for (int kk = 0; kk < C::PV_STEPS; ++kk)
-        umma_ts<false>(tmem + 256 + D, tmem + 128 + kk * 8, desc_add(vQ0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
-                       (i == 0 && kk == 0) ? 0u : 1u);
+        umma_ts<false>(tmem + 256 + D, tmem + 128 + packed_col(kk), desc_add(vQ0, off + mnmajor_off<16>(kk)),
+                       C::IDESC_ACC, (i == 0 && kk == 0) ? 0u : 1u);
       tc_commit(bar(kBarO));
     };
 
@@ -371,27 +420,21 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
         // every (key, query) pair of the tile visible: no test per column
         const bool full = j0 + kBN - 1 <= i0 && i0 + kBM - 1 < a.L &&
                           (j0 >= i0 + kBM - a.window || j0 + kBN - 1 < a.n_sink);
-        uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
-        if (!full) visible_words(s_key - i0, t_hi - i0, -1, vw);
         uint32_t sr[64], dr[64];
         tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
         tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
         uint32_t pw[32], dw[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float p[2], ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 64 * half + c + e;
-            const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - L_s[col]);
-            p[e] = word_bit(vw, col) ? pe : 0.f;
-            ds[e] = p[e] * (__uint_as_float(dr[c + e]) - D_s[col]);
-          }
-          pw[c / 2] = pack_bf16x2(p[0], p[1]);
-          dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
+        if (full) {
+          dkdv_elementwise<false>(sr, dr, D_s, L_s, a.scale_log2, nullptr, 64 * half, pw, dw);
+        } else {
+          uint32_t vw[4];
+          visible_words(s_key - i0, t_hi - i0, -1, vw);
+          dkdv_elementwise<true>(sr, dr, D_s, L_s, a.scale_log2, vw, 64 * half, pw, dw);
         }
-        tmem_st32(tmem + lane_off + 32 * half, pw);
-        tmem_st32(tmem + lane_off + 128 + 32 * half, dw);
+        // packed into the first half of this warpgroup's own columns: the other
+        // warpgroup may still be reading its S^T and dP^T columns
+        tmem_st32(tmem + lane_off + 64 * half, pw);
+        tmem_st32(tmem + lane_off + 128 + 64 * half, dw);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -428,8 +471,16 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
 }
 
 // ------------------------------------------------------------------ dQ
+// Roles as in the dK/dV kernel: warps 0-7 the element-wise step (thread = TMEM lane
+// = query row, warpgroup 0 on key columns 0-63, warpgroup 1 on 64-127), warp 8
+// (lane 0) TMA and MMA.  Per key tile j the producer waits for dS(j), issues
+// dQ += dS K and right behind it S and dP of key tile j + 1, and, once the
+// accumulation of j has read K(j), requests K and V of tile j + 2 into that buffer.
+constexpr int kDqThreads = 288;
+constexpr int kDqProducerWarp = 8;
+
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     swa_bwd_dq_kernel(const __grid_constant__ BwdArgs ba, const __grid_constant__ CUtensorMap tq,
                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                       const __grid_constant__ CUtensorMap tdo) {
@@ -443,6 +494,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sQ = base + C::OFF_T, sdO = sQ + C::TILE, sK = sdO + C::TILE, sV = sK + C::TILE;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
 
   const int tiles = (a.L + kBM - 1) / kBM;
   const int qt = blockIdx.x % tiles;
@@ -453,11 +505,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   decode_tile(a, nullptr, nullptr, b * tiles + qt, x);
 
   if (tid == 0) {
-    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i == kBarP ? kBwdThreads : 1);
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i == kBarP ? kEwThreads : 1);
     fence_mbar_init();
   }
-  __syncwarp();
-  if (tid < 32) {
+  if (warp == 0) {
     tmem_alloc(smem_u32(tmem_ptr), 512);
     tmem_relinquish();
   }
@@ -465,129 +516,143 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const int r = tid & 127;                            // TMEM lane (query row) of this thread
-  const int half = tid >> 7;                          // key columns 64 half .. 64 half + 63
-  const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
   const size_t row_base = static_cast<size_t>(b) * a.L;
-  const int t = x.m0 + r;                             // this thread's query row
-
+  const int n = x.n_tiles;
   bool ok = true;
-  int issued = 0;                                     // key tiles whose K, V were requested
-  auto issue = [&](int jj) {                          // thread 0: K, V of key tile step jj
-    const int buf = jj & 1, n0 = tile_n0(x, jj);
-    mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
-    load_tile<D>(sK + 2 * buf * C::TILE, &tk, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
-    load_tile<D>(sV + 2 * buf * C::TILE, &tv, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
-  };
-  if (tid == 0) {
-    mbar_expect_tx(bar(kBarA), 2 * C::TILE);
-    load_tile<D>(sQ, &tq, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
-    load_tile<D>(sdO, &tdo, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
-    issue(0);
-    issued = 1;
-  }
-  float dt = 0.f, l2 = 0.f;
-  if (t < a.L) {
-    const size_t off = ((row_base + t) * a.Hq + h) * D;
-    dt = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + off, static_cast<const __nv_bfloat16*>(ba.out) + off);
-    l2 = ba.lse[(static_cast<size_t>(b) * a.Hq + h) * a.L + t] * 1.4426950408889634f;
-  }
-  int j = 0;
-  for (; ok && j < x.n_tiles; ++j) {
-    const int n0 = tile_n0(x, j), buf = j & 1;
-    const uint32_t cK = sK + 2 * buf * C::TILE, cV = sV + 2 * buf * C::TILE;
-    if (tid == 0) {
-      // the next key tile's K, V: its buffer's last readers finished with step j-1
-      if (j + 1 < x.n_tiles) {
-        issue(j + 1);
-        issued = j + 2;
-      }
-      ok = (j > 0 || bwd_wait(bar(kBarA), 0, a)) && bwd_wait(bar(kBarB + buf), (j >> 1) & 1, a);
-      if (ok) {
-        tc_fence_after();
+
+  if (warp == kDqProducerWarp) {
+    if (lane == 0) {
+      // one descriptor per operand array, stepped by offsets (buffer, k-step)
+      const uint64_t dQ0 = kmajor_desc<4>(sQ, kBM, 0), ddO0 = kmajor_desc<4>(sdO, kBM, 0);
+      const uint64_t dK0 = kmajor_desc<4>(sK, kBN, 0), dV0 = kmajor_desc<4>(sV, kBN, 0);
+      const uint64_t vK0 = v_desc<false, 16>(sK, 0);
+      auto load_kv = [&](int jj) {                    // K, V of key tile step jj into buffer jj & 1
+        const int buf = jj & 1, n0 = tile_n0(x, jj);
+        mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
+        load_tile<D>(sK + 2 * buf * C::TILE, &tk, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
+        load_tile<D>(sV + 2 * buf * C::TILE, &tv, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
+      };
+      auto scores = [&](int jj) {                     // S = Q K^T, dP = dO V^T of key tile step jj
+        const uint32_t off = 2 * (jj & 1) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem, kmajor_desc<4>(sQ, kBM, kk), kmajor_desc<4>(cK, kBN, kk), C::IDESC_SS,
-                         kk > 0 ? 1u : 0u);
+          umma_ss<false>(tmem, desc_add(dQ0, kmajor_off<4, kBM>(kk)), desc_add(dK0, off + kmajor_off<4, kBN>(kk)),
+                         C::IDESC_SS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem + 128, kmajor_desc<4>(sdO, kBM, kk), kmajor_desc<4>(cV, kBN, kk), C::IDESC_SS,
-                         kk > 0 ? 1u : 0u);
+          umma_ss<false>(tmem + 128, desc_add(ddO0, kmajor_off<4, kBM>(kk)), desc_add(dV0, off + kmajor_off<4, kBN>(kk)),
+                         C::IDESC_SS, kk > 0 ? 1u : 0u);
         tc_commit(bar(kBarS));
-      }
-    }
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarS), j & 1, a)))) break;
-    tc_fence_after();
-    // dS of this query row over this warpgroup's 64 key columns, written over S
-    {
-      uint32_t vw[4] = {~0u, ~0u, ~0u, ~0u};
-      if (tile_needs_mask(x, j, a.window) || x.m1 - x.m0 != kBM - 1) {
-        // keys t - window + 1 .. t and the sinks below min(n_sink, t + 1); nothing past the end
-        if (t < a.L) visible_words(t - a.window + 1 - n0, t - n0, min(a.n_sink, t + 1) - 1 - n0, vw);
-        else vw[0] = vw[1] = vw[2] = vw[3] = 0u;
-      }
-      uint32_t sr[64], dr[64];
-      tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
-      tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
-      uint32_t dw[32];
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        float ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 64 * half + c + e;
-          const float pe = ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - l2);
-          const float p = word_bit(vw, col) ? pe : 0.f;
-          ds[e] = p * (__uint_as_float(dr[c + e]) - dt);
-        }
-        dw[c / 2] = pack_bf16x2(ds[0], ds[1]);
-      }
-      tmem_st32(tmem + lane_off + 32 * half, dw);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(bar(kBarP));
-    if (tid == 0) {
-      if ((ok = bwd_wait(bar(kBarP), j & 1, a))) {
-        tc_fence_after();
+      };
+      auto accumulate = [&](int jj) {                 // dQ += dS K of key tile step jj
+        const uint32_t off = 2 * (jj & 1) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256, tmem + kk * 8, v_desc<false, 16>(cK, kk), C::IDESC_ACC,
-                         (j == 0 && kk == 0) ? 0u : 1u);
+          umma_ts<false>(tmem + 256, tmem + packed_col(kk), desc_add(vK0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+                         (jj == 0 && kk == 0) ? 0u : 1u);
         tc_commit(bar(kBarO));
+      };
+      int issued = 0, waited = 0;                     // K/V loads requested / their arrivals seen
+      mbar_expect_tx(bar(kBarA), 2 * C::TILE);
+      load_tile<D>(sQ, &tq, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
+      load_tile<D>(sdO, &tdo, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
+      load_kv(0);
+      issued = 1;
+      if (n > 1) {
+        load_kv(1);
+        issued = 2;
+      }
+      if ((ok = bwd_wait(bar(kBarA), 0, a) && bwd_wait(bar(kBarB), 0, a))) {
+        waited = 1;
+        tc_fence_after();
+        scores(0);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        if (!(ok = bwd_wait(bar(kBarP), j & 1, a))) break;      // dS(j) written
+        tc_fence_after();
+        accumulate(j);
+        if (j + 1 < n) {
+          if (!(ok = bwd_wait(bar(kBarB + ((j + 1) & 1)), ((j + 1) >> 1) & 1, a))) break;
+          waited = j + 2;
+          tc_fence_after();
+          scores(j + 1);
+        }
+        if (j + 2 < n) {
+          // the accumulation of j read K from buffer j & 1
+          if (!(ok = bwd_wait(bar(kBarO), j & 1, a))) break;
+          load_kv(j + 2);
+          issued = j + 3;
+        }
+      }
+      // every product is issued: the drain barrier's only phase completes when all are done
+      tc_commit(bar(kBarDrain));
+      if (!ok) {
+        // let everything this thread started finish before the CTA releases its memory
+        bwd_wait(bar(kBarDrain), 0, a);
+        bwd_wait(bar(kBarA), 0, a);
+        for (int i = waited; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
       }
     }
     __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarO), j & 1, a)))) break;
-  }
-  if (!ok && tid == 0) {
-    tc_commit(bar(kBarDrain));
-    bwd_wait(bar(kBarDrain), 0, a);
-    bwd_wait(bar(kBarA), 0, a);
-    for (int i = j; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
-  }
-  __syncwarp();
-  tc_fence_after();
-  if (__all_sync(0xffffffffu, ok)) {        // warp-uniform: the TMEM loads are warp-collective
-    const bool row_ok = t < a.L;
-    float* dq = ba.dq + ((row_base + (row_ok ? t : 0)) * a.Hq + h) * D;
+  } else {
+    const int r = tid & 127;                          // TMEM lane (query row) of this thread
+    const int half = tid >> 7;                        // key columns 64 half .. 64 half + 63
+    const uint32_t lane_off = static_cast<uint32_t>((r >> 5) * 32) << 16;
+    const int t = x.m0 + r;                           // this thread's query row
+    float dt = 0.f, l2 = 0.f;
+    if (t < a.L) {
+      const size_t off = ((row_base + t) * a.Hq + h) * D;
+      dt = row_dot<D>(static_cast<const __nv_bfloat16*>(ba.dout) + off, static_cast<const __nv_bfloat16*>(ba.out) + off);
+      l2 = ba.lse[(static_cast<size_t>(b) * a.Hq + h) * a.L + t] * 1.4426950408889634f;
+    }
+    for (int j = 0; j < n; ++j) {
+      const int n0 = tile_n0(x, j);
+      if (!(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarS), j & 1, a)))) break;
+      tc_fence_after();
+      // dS of this query row over this warpgroup's 64 key columns, written over S
+      {
+        uint32_t sr[64], dr[64];
+        tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
+        tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
+        uint32_t dw[32];
+        if (tile_needs_mask(x, j, a.window) || x.m1 - x.m0 != kBM - 1) {
+          // keys t - window + 1 .. t and the sinks below min(n_sink, t + 1); nothing past the end
+          uint32_t vw[4] = {0u, 0u, 0u, 0u};
+          if (t < a.L) visible_words(t - a.window + 1 - n0, t - n0, min(a.n_sink, t + 1) - 1 - n0, vw);
+          dq_elementwise<true>(sr, dr, dt, l2, a.scale_log2, vw, 64 * half, dw);
+        } else {
+          dq_elementwise<false>(sr, dr, dt, l2, a.scale_log2, nullptr, 64 * half, dw);
+        }
+        // packed into the first half of this warpgroup's own columns (see packed_col)
+        tmem_st32(tmem + lane_off + 64 * half, dw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+    }
+    // all products done (a single-phase barrier: no parity can be confused with another)
+    ok = __all_sync(0xffffffffu, ok && bwd_wait(bar(kBarDrain), 0, a));
+    tc_fence_after();
+    if (ok) {                                 // warp-uniform: the TMEM loads are warp-collective
+      const bool row_ok = t < a.L;
+      float* dq = ba.dq + ((row_base + (row_ok ? t : 0)) * a.Hq + h) * D;
 #pragma unroll 1
-    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
-      uint32_t r[32];
-      tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, r);
-      if (!row_ok) continue;
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {   // this warpgroup's half of d
+        uint32_t rr[32];
+        tmem_ld32_wait(tmem + lane_off + 256 + 32 * c, rr);
+        if (!row_ok) continue;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(dq + 32 * c + i) =
-            make_float4(__uint_as_float(r[i]) * a.scale, __uint_as_float(r[i + 1]) * a.scale,
-                        __uint_as_float(r[i + 2]) * a.scale, __uint_as_float(r[i + 3]) * a.scale);
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dq + 32 * c + i) =
+              make_float4(__uint_as_float(rr[i]) * a.scale, __uint_as_float(rr[i + 1]) * a.scale,
+                          __uint_as_float(rr[i + 2]) * a.scale, __uint_as_float(rr[i + 3]) * a.scale);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid < 32) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 template <int D>
@@ -610,7 +675,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
     int n1 = 0, n2 = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, swa_bwd_dkdv_kernel<D>, kDkdvThreads, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kBwdThreads, C::SMEM_BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kDqThreads, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (n1 != 1 || n2 != 1) return cudaErrorNotSupported;
     checked = 1;
@@ -622,7 +687,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
   swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kDkdvThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kBwdThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
+  swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kDqThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   return cudaGetLastError();
 }
 
