@@ -33,8 +33,8 @@
 //
 // TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
 // written over columns 0-31 and 64-95 of each, every warpgroup within the columns
-// it read), dV 256.., dK 256+d..; (dQ kernel): S 0-127 (dS packed the same way),
-// dP 128-255, dQ 256...
+// it read), dV 256.., dK 256+d..; (dQ kernel): S 0-127, dP 128-255, dQ 256..,
+// dS packed at 384-415 and 448-479.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -82,6 +82,7 @@ constexpr int kBarO = 5;      // accumulation products done
 constexpr int kBarRow = 6;    // dK/dV kernel: row data (D, lse) of even iterations staged
 constexpr int kBarDrain = 7;
 constexpr int kBarRow2 = 8;   // dK/dV kernel: row data of odd iterations staged
+constexpr int kBarRead = 6;   // dQ kernel: every element-wise thread has read S and dP
 
 __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const PrefillArgs& a) {
   for (int i = 0; i < 256; ++i)
@@ -473,9 +474,13 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
 // ------------------------------------------------------------------ dQ
 // Roles as in the dK/dV kernel: warps 0-7 the element-wise step (thread = TMEM lane
 // = query row, warpgroup 0 on key columns 0-63, warpgroup 1 on 64-127), warp 8
-// (lane 0) TMA and MMA.  Per key tile j the producer waits for dS(j), issues
-// dQ += dS K and right behind it S and dP of key tile j + 1, and, once the
-// accumulation of j has read K(j), requests K and V of tile j + 2 into that buffer.
+// (lane 0) TMA and MMA.  dS goes to TMEM columns 384-511, apart from S and dP, so
+// the scores of key tile j + 1 are computed while the element-wise step of j runs:
+// the element-wise warps signal once they have read S(j) and dP(j) (barrier R), the
+// producer then issues S and dP of j + 1, and after dS(j) is written, dQ += dS K.
+// An element-wise warp writes dS(j) only after the accumulation of j - 1 has read
+// dS(j - 1).  Once the accumulation of j has read K(j), K and V of tile j + 2 are
+// requested into that buffer.
 constexpr int kDqThreads = 288;
 constexpr int kDqProducerWarp = 8;
 
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   decode_tile(a, nullptr, nullptr, b * tiles + qt, x);
 
   if (tid == 0) {
-    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i == kBarP ? kEwThreads : 1);
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i == kBarP || i == kBarRead ? kEwThreads : 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -516,6 +521,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
+  const uint32_t tmem_ds = tmem + 384;                // packed dS (see packed_col)
   const size_t row_base = static_cast<size_t>(b) * a.L;
   const int n = x.n_tiles;
   bool ok = true;
@@ -548,7 +554,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t off = 2 * (jj & 1) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256, tmem + packed_col(kk), desc_add(vK0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+          umma_ts<false>(tmem + 256, tmem_ds + packed_col(kk), desc_add(vK0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
                          (jj == 0 && kk == 0) ? 0u : 1u);
         tc_commit(bar(kBarO));
       };
@@ -568,15 +574,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         scores(0);
       }
       for (int j = 0; ok && j < n; ++j) {
-        if (!(ok = bwd_wait(bar(kBarP), j & 1, a))) break;      // dS(j) written
-        tc_fence_after();
-        accumulate(j);
         if (j + 1 < n) {
-          if (!(ok = bwd_wait(bar(kBarB + ((j + 1) & 1)), ((j + 1) >> 1) & 1, a))) break;
+          // S(j) and dP(j) have been read: their columns take the scores of j + 1
+          if (!(ok = bwd_wait(bar(kBarRead), j & 1, a) &&
+                     bwd_wait(bar(kBarB + ((j + 1) & 1)), ((j + 1) >> 1) & 1, a)))
+            break;
           waited = j + 2;
           tc_fence_after();
           scores(j + 1);
         }
+        if (!(ok = bwd_wait(bar(kBarP), j & 1, a))) break;      // dS(j) written
+        tc_fence_after();
+        accumulate(j);
         if (j + 2 < n) {
           // the accumulation of j read K from buffer j & 1
           if (!(ok = bwd_wait(bar(kBarO), j & 1, a))) break;
@@ -614,6 +623,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         uint32_t sr[64], dr[64];
         tmem_ld64_wait(tmem + lane_off + 64 * half, sr);
         tmem_ld64_wait(tmem + lane_off + 128 + 64 * half, dr);
+        tc_fence_before();
+        mbar_arrive(bar(kBarRead));                   // S(j), dP(j) read
         uint32_t dw[32];
         if (tile_needs_mask(x, j, a.window) || x.m1 - x.m0 != kBM - 1) {
           // keys t - window + 1 .. t and the sinks below min(n_sink, t + 1); nothing past the end
@@ -623,8 +634,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         } else {
           dq_elementwise<false>(sr, dr, dt, l2, a.scale_log2, nullptr, 64 * half, dw);
         }
-        // packed into the first half of this warpgroup's own columns (see packed_col)
-        tmem_st32(tmem + lane_off + 64 * half, dw);
+        // the accumulation of j - 1 has read dS(j - 1) before it is overwritten
+        if (j > 0 && !(ok = __all_sync(0xffffffffu, bwd_wait(bar(kBarO), (j - 1) & 1, a)))) break;
+        tc_fence_after();
+        tmem_st32(tmem_ds + lane_off + 64 * half, dw);
       }
       tmem_wait_st();
       tc_fence_before();
