@@ -73,6 +73,20 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_ACC = make_idesc(1u, kBM, D, true);     // 128 x d accumulators
 };
 
+// dQ kernel layout: Q, dO, three K buffers, two V buffers (K is read by both the score
+// and the accumulation products, so it is kept one key tile longer), then barriers.
+template <int D>
+struct DqCfg : BwdCfg<D> {
+  using B = BwdCfg<D>;
+  static constexpr int OFF_K = 2 * B::TILE;
+  static constexpr int OFF_V = 5 * B::TILE;
+  static constexpr int OFF_BAR = 7 * B::TILE;
+  static constexpr int NBAR = 11;
+  static constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
+  static constexpr int SMEM_USED = OFF_TMEMPTR + 16 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_USED > 119808 ? SMEM_USED : 119808;
+};
+
 // barrier indices
 constexpr int kBarA = 0;      // K,V (dK/dV kernel) or Q,dO (dQ kernel): loaded once
 constexpr int kBarB = 1;      // the per-iteration tile pair, buffers 0 and 1 (kBarB, kBarB + 1)
@@ -83,6 +97,7 @@ constexpr int kBarRow = 6;    // dK/dV kernel: row data (D, lse) of even iterati
 constexpr int kBarDrain = 7;
 constexpr int kBarRow2 = 8;   // dK/dV kernel: row data of odd iterations staged
 constexpr int kBarRead = 6;   // dQ kernel: every element-wise thread has read S and dP
+constexpr int kBarKf = 8;     // dQ kernel: K buffers 0-2 loaded (kBarB, kBarB + 1: V buffers)
 
 __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const PrefillArgs& a) {
   for (int i = 0; i < 256; ++i)
@@ -479,8 +494,9 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
 // the element-wise warps signal once they have read S(j) and dP(j) (barrier R), the
 // producer then issues S and dP of j + 1, and after dS(j) is written, dQ += dS K.
 // An element-wise warp writes dS(j) only after the accumulation of j - 1 has read
-// dS(j - 1).  Once the accumulation of j has read K(j), K and V of tile j + 2 are
-// requested into that buffer.
+// dS(j - 1).  K is kept in three buffers and V in two: V of tile j + 2 is requested
+// as soon as the scores of j have been read, K of tile j + 3 once the accumulation
+// of j has read K(j), so both arrive a key tile or more before their score products.
 constexpr int kDqThreads = 288;
 constexpr int kDqProducerWarp = 8;
 
@@ -489,14 +505,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     swa_bwd_dq_kernel(const __grid_constant__ BwdArgs ba, const __grid_constant__ CUtensorMap tq,
                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                       const __grid_constant__ CUtensorMap tdo) {
-  using C = BwdCfg<D>;
+  using C = DqCfg<D>;
   const PrefillArgs& a = ba.pa;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8 * i; };
-  const uint32_t sQ = base + C::OFF_T, sdO = sQ + C::TILE, sK = sdO + C::TILE, sV = sK + C::TILE;
+  const uint32_t sQ = base + C::OFF_T, sdO = sQ + C::TILE, sK = base + C::OFF_K, sV = base + C::OFF_V;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEMPTR);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -532,65 +548,72 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const uint64_t dQ0 = kmajor_desc<4>(sQ, kBM, 0), ddO0 = kmajor_desc<4>(sdO, kBM, 0);
       const uint64_t dK0 = kmajor_desc<4>(sK, kBN, 0), dV0 = kmajor_desc<4>(sV, kBN, 0);
       const uint64_t vK0 = v_desc<false, 16>(sK, 0);
-      auto load_kv = [&](int jj) {                    // K, V of key tile step jj into buffer jj & 1
-        const int buf = jj & 1, n0 = tile_n0(x, jj);
-        mbar_expect_tx(bar(kBarB + buf), 2 * C::TILE);
-        load_tile<D>(sK + 2 * buf * C::TILE, &tk, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
-        load_tile<D>(sV + 2 * buf * C::TILE, &tv, bar(kBarB + buf), kvh, static_cast<int>(row_base) + n0);
+      auto load_k = [&](int jj) {                     // K of key tile step jj into K buffer jj % 3
+        const int buf = jj % 3;
+        mbar_expect_tx(bar(kBarKf + buf), C::TILE);
+        load_tile<D>(sK + buf * C::TILE, &tk, bar(kBarKf + buf), kvh, static_cast<int>(row_base) + tile_n0(x, jj));
       };
+      auto load_v = [&](int jj) {                     // V of key tile step jj into V buffer jj & 1
+        const int buf = jj & 1;
+        mbar_expect_tx(bar(kBarB + buf), C::TILE);
+        load_tile<D>(sV + buf * C::TILE, &tv, bar(kBarB + buf), kvh, static_cast<int>(row_base) + tile_n0(x, jj));
+      };
+      auto wait_k = [&](int jj) { return bwd_wait(bar(kBarKf + jj % 3), (jj / 3) & 1, a); };
+      auto wait_v = [&](int jj) { return bwd_wait(bar(kBarB + (jj & 1)), (jj >> 1) & 1, a); };
       auto scores = [&](int jj) {                     // S = Q K^T, dP = dO V^T of key tile step jj
-        const uint32_t off = 2 * (jj & 1) * C::TILE;
+        const uint32_t offk = (jj % 3) * C::TILE, offv = (jj & 1) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem, desc_add(dQ0, kmajor_off<4, kBM>(kk)), desc_add(dK0, off + kmajor_off<4, kBN>(kk)),
+          umma_ss<false>(tmem, desc_add(dQ0, kmajor_off<4, kBM>(kk)), desc_add(dK0, offk + kmajor_off<4, kBN>(kk)),
                          C::IDESC_SS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk)
-          umma_ss<false>(tmem + 128, desc_add(ddO0, kmajor_off<4, kBM>(kk)), desc_add(dV0, off + kmajor_off<4, kBN>(kk)),
+          umma_ss<false>(tmem + 128, desc_add(ddO0, kmajor_off<4, kBM>(kk)), desc_add(dV0, offv + kmajor_off<4, kBN>(kk)),
                          C::IDESC_SS, kk > 0 ? 1u : 0u);
         tc_commit(bar(kBarS));
       };
       auto accumulate = [&](int jj) {                 // dQ += dS K of key tile step jj
-        const uint32_t off = 2 * (jj & 1) * C::TILE;
+        const uint32_t offk = (jj % 3) * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk)
-          umma_ts<false>(tmem + 256, tmem_ds + packed_col(kk), desc_add(vK0, off + mnmajor_off<16>(kk)), C::IDESC_ACC,
+          umma_ts<false>(tmem + 256, tmem_ds + packed_col(kk), desc_add(vK0, offk + mnmajor_off<16>(kk)), C::IDESC_ACC,
                          (jj == 0 && kk == 0) ? 0u : 1u);
         tc_commit(bar(kBarO));
       };
-      int issued = 0, waited = 0;                     // K/V loads requested / their arrivals seen
+      // loads requested / their arrivals seen, for K and for V
+      int issued_k = 0, issued_v = 0, waited_k = 0, waited_v = 0;
       mbar_expect_tx(bar(kBarA), 2 * C::TILE);
       load_tile<D>(sQ, &tq, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
       load_tile<D>(sdO, &tdo, bar(kBarA), h, static_cast<int>(row_base) + x.m0);
-      load_kv(0);
-      issued = 1;
-      if (n > 1) {
-        load_kv(1);
-        issued = 2;
-      }
-      if ((ok = bwd_wait(bar(kBarA), 0, a) && bwd_wait(bar(kBarB), 0, a))) {
-        waited = 1;
+      for (; issued_k < min(n, 3); ++issued_k) load_k(issued_k);
+      for (; issued_v < min(n, 2); ++issued_v) load_v(issued_v);
+      if ((ok = bwd_wait(bar(kBarA), 0, a) && wait_k(0) && wait_v(0))) {
+        waited_k = waited_v = 1;
         tc_fence_after();
         scores(0);
       }
       for (int j = 0; ok && j < n; ++j) {
         if (j + 1 < n) {
-          // S(j) and dP(j) have been read: their columns take the scores of j + 1
-          if (!(ok = bwd_wait(bar(kBarRead), j & 1, a) &&
-                     bwd_wait(bar(kBarB + ((j + 1) & 1)), ((j + 1) >> 1) & 1, a)))
-            break;
-          waited = j + 2;
+          // S(j) and dP(j) have been read, so the score products of j are done: V buffer
+          // j & 1 takes V of j + 2, and the score columns take the scores of j + 1
+          if (!(ok = bwd_wait(bar(kBarRead), j & 1, a))) break;
+          if (j + 2 < n) {
+            load_v(j + 2);
+            issued_v = j + 3;
+          }
+          if (!(ok = wait_k(j + 1) && wait_v(j + 1))) break;
+          waited_k = waited_v = j + 2;
           tc_fence_after();
           scores(j + 1);
         }
         if (!(ok = bwd_wait(bar(kBarP), j & 1, a))) break;      // dS(j) written
         tc_fence_after();
         accumulate(j);
-        if (j + 2 < n) {
-          // the accumulation of j read K from buffer j & 1
+        if (j + 3 < n) {
+          // the accumulation of j is the last reader of K buffer j % 3
           if (!(ok = bwd_wait(bar(kBarO), j & 1, a))) break;
-          load_kv(j + 2);
-          issued = j + 3;
+          load_k(j + 3);
+          issued_k = j + 4;
         }
       }
       // every product is issued: the drain barrier's only phase completes when all are done
@@ -599,7 +622,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // let everything this thread started finish before the CTA releases its memory
         bwd_wait(bar(kBarDrain), 0, a);
         bwd_wait(bar(kBarA), 0, a);
-        for (int i = waited; i < issued; ++i) bwd_wait(bar(kBarB + (i & 1)), (i >> 1) & 1, a);
+        for (int i = waited_k; i < issued_k; ++i) wait_k(i);
+        for (int i = waited_v; i < issued_v; ++i) wait_v(i);
       }
     }
     __syncwarp();
@@ -680,7 +704,8 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
   cudaError_t e = cudaFuncSetAttribute(swa_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(swa_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  static_assert(DqCfg<D>::SMEM_BYTES <= 232448, "shared memory budget");
+  e = cudaFuncSetAttribute(swa_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqCfg<D>::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // one CTA per SM (see SMEM_BYTES): refuse to launch if the occupancy says otherwise
   static int checked = 0;
@@ -688,7 +713,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
     int n1 = 0, n2 = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, swa_bwd_dkdv_kernel<D>, kDkdvThreads, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kDqThreads, C::SMEM_BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n2, swa_bwd_dq_kernel<D>, kDqThreads, DqCfg<D>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (n1 != 1 || n2 != 1) return cudaErrorNotSupported;
     checked = 1;
@@ -700,7 +725,7 @@ cudaError_t launch_bwd_impl(const BwdArgs& ba, const CUtensorMap& tq, const CUte
   swa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(g_kv), kDkdvThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kDqThreads, C::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
+  swa_bwd_dq_kernel<D><<<static_cast<unsigned>(g_q), kDqThreads, DqCfg<D>::SMEM_BYTES, stream>>>(ba, tq, tk, tv, tdo);
   return cudaGetLastError();
 }
 
