@@ -44,6 +44,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -213,13 +214,21 @@ def load_peaks():
         return dict(PEAKS_FALLBACK, source="fallback")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and with runs of white space collapsed."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(files=None) -> str:
-    """Hash of the kernel sources (all of them, or the named files of csrc/)."""
+    """Hash of the kernel sources (all of them, or the named files of csrc/).  Comments
+    and white space are left out, so editing a comment keeps a capture valid."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sink_aware_sliding_b200", "csrc")
     names = sorted(files) if files else sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h")))
     for name in names:
-        h.update(open(os.path.join(csrc, name), "rb").read())
+        h.update(_code_only(open(os.path.join(csrc, name), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -24,12 +24,14 @@
 // Visibility is tested only on edge tiles, through four 32-bit words per row built
 // from the row's visible column ranges (a separate code path for fully visible
 // tiles).  Every hand-off is an mbarrier with a bounded wait.  In both kernels a
-// ninth warp issues TMA and MMA, so the accumulation products of one iteration and
-// the score products of the next go out back to back and the element-wise warps
-// wait only for their scores; the tiles that change per iteration (Q and dO, or K
-// and V) are double-buffered and requested two iterations ahead.  The products and
-// the element-wise step of one iteration still run one after another (TMEM holds
-// one iteration's scores next to the accumulators).
+// ninth warp issues TMA and MMA, so the element-wise warps wait only for their
+// scores.  In the dK/dV kernel the accumulation products of one iteration and the
+// score products of the next go out back to back, Q and dO are double-buffered and
+// requested two iterations ahead, and the products and the element-wise step of one
+// iteration run one after another (TMEM holds one iteration's scores next to the
+// two accumulators).  In the dQ kernel dS has TMEM columns of its own, so the score
+// products of the next key tile run during the element-wise step; K is kept in
+// three buffers and V in two.
 //
 // TMEM (dK/dV kernel): S^T 0-127, dP^T 128-255 (P^T and dS^T, packed bf16, are
 // written over columns 0-31 and 64-95 of each, every warpgroup within the columns
@@ -49,7 +51,7 @@ namespace {
 
 using namespace prefill;
 
-constexpr int kEwThreads = 256;    // dK/dV kernel: the element-wise threads (warps 0-7)
+constexpr int kEwThreads = 256;    // the element-wise threads of both kernels (warps 0-7)
 
 template <int D>
 struct BwdCfg {
