@@ -169,7 +169,9 @@ __device__ __forceinline__ void window_step(const HybridArgs& a, int bh, int tid
   }
 }
 
-__global__ void __launch_bounds__(kHybThreads, 4) swa_hybrid_decode_kernel(const __grid_constant__ HybridArgs a) {
+// Five blocks per SM (48 registers, a few bytes spilled): measured 4% faster than
+// four (64 registers, no spill); six spill too much and are slower.
+__global__ void __launch_bounds__(kHybThreads, 5) swa_hybrid_decode_kernel(const __grid_constant__ HybridArgs a) {
   const int n_lin = a.B * a.H_l;
   if (static_cast<int>(blockIdx.x) < n_lin) {
     lin::decode_step(blockIdx.x, threadIdx.x, static_cast<const __nv_bfloat16*>(a.ql),
