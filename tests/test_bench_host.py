@@ -75,3 +75,22 @@ def test_reduce_max_over_two_gloo_ranks():
 
 def test_reduce_max_without_process_group_is_identity():
     assert bench.reduce_max(3.25) == 3.25
+
+
+def test_source_hash_ignores_comments_and_spacing():
+    """A comment or spacing edit keeps a DRAM-traffic capture valid; a code edit does not."""
+    code = "int f(int x) {\n  return x + 1;  // next\n}\n/* block\n comment */\n"
+    assert bench._code_only(code) == bench._code_only("int f(int x) { return x + 1; }")
+    assert bench._code_only(code) != bench._code_only("int f(int x) { return x + 2; }")
+
+
+def test_traffic_table_entries_name_existing_sources():
+    import json
+    t = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")))
+    csrc = os.path.join(os.path.dirname(bench.__file__), "sink_aware_sliding_b200", "csrc")
+    for name, e in t.items():
+        if name == "about":
+            continue
+        assert e["dram_bytes_per_launch"] > 0
+        for f in e["sources"]:
+            assert os.path.exists(os.path.join(csrc, f)), (name, f)
