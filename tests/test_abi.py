@@ -137,3 +137,40 @@ def test_based_linear_binding_checks_shapes(lib):
     with pytest.raises(ValueError):
         swa.swa_based_linear_decode(qd, qd, vd, torch.zeros(1, 2, 273, 64), torch.zeros(1, 2, 272),
                                     torch.zeros(1, 2, 64))
+
+
+def test_decode_ex_hybrid_and_backward_argument_checks(lib):
+    F = ctypes.c_float
+    Z = ctypes.c_size_t(0)
+
+    def dex(B=1, Hq=4, Hkv=2, d=128, W=64, S=4, scale=0.1, out_dtype=2):
+        return lib.swa_decode_ex(None, None, None, None, None, None, None, None, B, Hq, Hkv, d, W, S,
+                                 F(scale), out_dtype, None, Z, None)
+    assert dex(out_dtype=1) == swa.SWA_ERR_INVALID_ARG            # f32 inputs: no decode
+    assert dex(out_dtype=7) == swa.SWA_ERR_INVALID_ARG
+    assert dex(scale=0.0) == swa.SWA_ERR_INVALID_ARG
+    assert dex(Hq=3) == swa.SWA_ERR_INVALID_ARG
+    assert dex(B=0) == swa.SWA_OK
+    assert dex() == swa.SWA_ERR_INVALID_ARG                       # null tensors
+
+    def hyb(B=1, Hq=4, Hkv=2, d=64, W=128, S=0, scale=0.125, H_l=2, dk=16, dv=64, scale_l=0.25):
+        return lib.swa_hybrid_decode(None, None, None, None, None, None, None, None, None, None,
+                                     B, Hq, Hkv, d, W, S, F(scale), None, None, None, None, None, None,
+                                     H_l, dk, dv, F(scale_l), None)
+    assert hyb(d=128) == swa.SWA_ERR_UNSUPPORTED                  # the window branch is d = 64 only
+    assert hyb(W=600) == swa.SWA_ERR_UNSUPPORTED                  # window + sinks above 512 keys
+    assert hyb(dk=8) == swa.SWA_ERR_UNSUPPORTED
+    assert hyb(scale_l=0.0) == swa.SWA_ERR_INVALID_ARG
+    assert hyb(Hq=3) == swa.SWA_ERR_INVALID_ARG
+    assert hyb(H_l=0) == swa.SWA_ERR_INVALID_ARG
+    assert hyb(B=0) == swa.SWA_OK
+    assert hyb() == swa.SWA_ERR_INVALID_ARG                       # null tensors
+
+    def bwd(B=1, Hq=4, Hkv=2, L=16, d=128, W=8, S=4, scale=0.1):
+        return lib.swa_bwd(None, None, None, None, None, None, None, None, None, B, Hq, Hkv, L, d, W, S,
+                           F(scale), None)
+    assert bwd(d=96) == swa.SWA_ERR_UNSUPPORTED
+    assert bwd(Hq=3) == swa.SWA_ERR_INVALID_ARG
+    assert bwd(W=0) == swa.SWA_ERR_INVALID_ARG
+    assert bwd(L=0) == swa.SWA_OK
+    assert bwd() == swa.SWA_ERR_INVALID_ARG                       # null tensors
